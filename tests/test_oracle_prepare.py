@@ -1,0 +1,296 @@
+"""Pins of the oracle's preparation steps and GEMM reference against the
+mathematics: closed forms, invariants, grid identities and brute force.  Each
+test is chosen so that a plausible slip in the oracle (a dropped factor, a
+wrong index, swapped nibbles, the unquantised backbone used for the residual)
+fails at least one of them."""
+import numpy as np
+import pytest
+
+import oracle
+from activation_sparsity_prep_b200 import workloads as wl
+
+F32 = np.float32
+
+
+def _bf16(a):
+    return wl.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+# -------------------------------------------------------------- RMSNorm ----
+
+@pytest.mark.parametrize("c", [1.0, -3.5, 0.0078125, 96.0])
+@pytest.mark.parametrize("K", [256, 768, 4096])
+def test_rmsnorm_constant_row_closed_form(c, K):
+    x = _bf16(np.full((1, K), c))
+    cv = float(wl.bf16_bits_to_f32(x)[0, 0])
+    y = oracle.normalize(x, wl.gamma_ones(K), 1e-6)
+    want = cv / np.sqrt(cv * cv + 1e-6)
+    ulp = np.spacing(np.float32(abs(want)))
+    assert np.all(np.abs(y.astype(np.float64) - want) <= 2 * ulp)
+
+
+def test_rmsnorm_matches_fp64_and_applies_gamma():
+    X = wl.activation("laplace_outlier", 9, 0, 8, 4096)
+    g = wl.gamma_random(9, 0, 4096)
+    y = oracle.normalize(X, g, 1e-6)
+    x64 = wl.bf16_bits_to_f32(X).astype(np.float64)
+    g64 = wl.bf16_bits_to_f32(g).astype(np.float64)
+    y64 = x64 / np.sqrt((x64 ** 2).mean(axis=1, keepdims=True) + 1e-6) * g64
+    rel = np.abs(y - y64) / np.maximum(np.abs(y64), 1e-30)
+    assert rel.max() < 2e-6
+    # gamma = NULL means no normalisation at all
+    assert np.array_equal(oracle.normalize(X, None, 1e-6), wl.bf16_bits_to_f32(X))
+
+
+def test_rms_sum_uses_the_stated_lane_order():
+    """x_0 = 2^14 (square 2^28, ulp 32) and two chunks of 1.25 (squares
+    1.5625) in chunks 1 and 3.  Strided chunk-to-lane assignment puts the
+    chunks in lanes 1 and 3 (12.5 each); the butterfly joins lanes 1 and 3
+    (25) before they meet lane 0, and 2^28 + 25 rounds to 2^28 + 32.  A
+    sequential sum, contiguous lanes or a linear lane sum all lose the small
+    terms one at a time and give 2^28."""
+    K = 512
+    x = np.zeros(K, dtype=np.float32)
+    x[0] = 2.0 ** 14
+    x[8:16] = 1.25
+    x[24:32] = 1.25
+    S_expect = np.float32(2.0 ** 28 + 32)
+    ms = np.float32(S_expect / np.float32(K))
+    rinv = np.float32(1) / np.sqrt(np.float32(ms + np.float32(1e-6)))
+    S_seq = np.float32(2.0 ** 28)
+    rinv_seq = np.float32(1) / np.sqrt(np.float32(np.float32(S_seq / np.float32(K)) + np.float32(1e-6)))
+    assert rinv != rinv_seq
+    got = oracle.rms_rinv(_bf16(x), 1e-6)
+    assert got == rinv
+
+
+# ------------------------------------------------------------------ mask ---
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (4, 8), (3, 4), (1, 8)])
+def test_mask_exact_n_per_group_and_bruteforce_sort(n, m):
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((7, 64)).astype(np.float32)
+    y[:, ::3] = np.round(y[:, ::3])          # plenty of ties
+    y[0, :8] = 0.0
+    y[1, :4] = [-0.0, 0.0, -0.0, 0.0]
+    keep = oracle.mask(y, n, m)
+    g = keep.reshape(7, -1, m)
+    assert np.all(g.sum(axis=2) == n)
+    for i in range(7):
+        for s in range(0, 64, m):
+            a = np.abs(y[i, s:s + m])
+            order = np.argsort(-a, kind="stable")          # ties -> lower index first
+            want = np.zeros(m, dtype=np.uint8)
+            want[order[:n]] = 1
+            assert np.array_equal(keep[i, s:s + m], want)
+            assert a[keep[i, s:s + m] == 1].max() == a.max()
+
+
+# ---------------------------------------------------------- quantisers -----
+
+def _grid_tensor_nvfp4(rng, R, K, j, sparse24=False):
+    """T on the NVFP4 grid: T = val * e0 * 2^j with one element equal to
+    6 * 448 * 2^j so that the tensor amax is exactly 2688 * 2^j.  With
+    ``sparse24`` positions 2 and 3 of every group of 4 are zero and each
+    block's amax element sits at a kept position."""
+    vals = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    e4 = oracle.e4m3_decode(np.arange(0x08, 0x7F, dtype=np.uint8)).astype(np.float64)
+    T = np.zeros((R, K))
+    kept = np.array([p for p in range(16) if (not sparse24) or p % 4 < 2])
+    for i in range(R):
+        for b in range(K // 16):
+            e0 = rng.choice(e4)
+            v = rng.choice(vals, 16) * rng.choice([-1, 1], 16)
+            if sparse24:
+                v[np.arange(16) % 4 >= 2] = 0.0
+            v[rng.choice(kept)] = 6.0 * rng.choice([-1, 1])    # block amax = 6 e0
+            T[i, b * 16:(b + 1) * 16] = v * e0 * 2.0 ** j
+    T[0, :16] = 0
+    T[0, 1] = 6 * 448 * 2.0 ** j
+    return T.astype(np.float32)
+
+
+@pytest.mark.parametrize("j", [-12, 0, 5])
+def test_nvfp4_identity_on_grid(j):
+    rng = np.random.default_rng(100 + j)
+    T = _grid_tensor_nvfp4(rng, 5, 128, j)
+    q = oracle.quantize(T, "nvfp4", want_D=True)
+    assert q.tscale == F32(2.0 ** j)
+    assert np.array_equal(q.D, T)
+    # codes decode to the right elements: even k in the low nibble
+    lo = q.codes & 15
+    hi = q.codes >> 4
+    dec = np.empty_like(T)
+    dec[:, 0::2] = oracle.e2m1_decode(lo)
+    dec[:, 1::2] = oracle.e2m1_decode(hi)
+    sc = np.repeat(oracle.e4m3_decode(q.scales), 16, axis=1)
+    assert np.array_equal((dec * sc * q.tscale).astype(np.float32), T)
+
+
+def test_mxfp4_identity_on_grid():
+    rng = np.random.default_rng(7)
+    vals = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    R, K = 3, 128
+    T = np.zeros((R, K))
+    for i in range(R):
+        for b in range(K // 32):
+            s = 2.0 ** rng.integers(-20, 20)
+            v = rng.choice(vals, 32) * rng.choice([-1, 1], 32)
+            v[rng.integers(32)] = rng.choice([4.0, 6.0])        # amax in {4,6} * s
+            T[i, b * 32:(b + 1) * 32] = v * s
+    T = T.astype(np.float32)
+    q = oracle.quantize(T, "mxfp4", want_D=True)
+    assert q.tscale == 1.0
+    assert np.array_equal(q.D, T)
+
+
+def test_nvfp4_scale_and_code_bounds():
+    """Away from the grid: the block scale is the E4M3 rounding of
+    amax_block * G_enc / 6, and each code is the nearest E2M1 value of
+    T * G_enc / e (checked with independent float64 arithmetic)."""
+    X = wl.activation("laplace_outlier", 11, 0, 4, 512)
+    T = wl.bf16_bits_to_f32(X)
+    q = oracle.quantize(T, "nvfp4", want_D=True)
+    A = np.abs(T).max().astype(np.float64)
+    assert abs(float(q.tscale) * 2688 - A) <= A * 2 ** -23
+    genc = 2688.0 / A
+    e = oracle.e4m3_decode(q.scales).astype(np.float64)
+    bmax = np.abs(T).reshape(4, -1, 16).max(axis=2).astype(np.float64)
+    target = bmax * genc / 6
+    # e is one of the two E4M3 neighbours of the target and the nearer one
+    allv = oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8)).astype(np.float64)
+    for t, ev in zip(target.ravel(), e.ravel()):
+        assert abs(ev - t) <= np.abs(allv - t).min() * (1 + 1e-6) + 1e-12
+    dec = np.empty(T.shape)
+    dec[:, 0::2] = oracle.e2m1_decode(q.codes & 15)
+    dec[:, 1::2] = oracle.e2m1_decode(q.codes >> 4)
+    x = T.astype(np.float64) * genc / np.repeat(e, 16, axis=1)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    ok = np.abs(np.abs(dec) - np.minimum(np.abs(x), 6.0)) <= \
+        np.min(np.abs(np.minimum(np.abs(x), 6.0)[..., None] - grid), axis=-1) + 1e-6
+    assert ok.all()
+
+
+# ------------------------------------------------------------- prepare -----
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (4, 8)])
+def test_prepare_reconstruction_exact(fmt, n, m):
+    """y == fl(D_b + r) bitwise: the residual is taken against the
+    dequantised backbone and the subtraction is exact (Sterbenz)."""
+    X = wl.activation("laplace_outlier", 12, 0, 6, 1024)
+    P = oracle.prepare(X, wl.gamma_ones(1024), 1e-6, n, m, fmt, keep_intermediates=True)
+    blk = 16 if fmt == "nvfp4" else 32
+    dec = np.empty(P.y.shape, dtype=np.float32)
+    dec[:, 0::2] = oracle.e2m1_decode(P.bb.codes & 15)
+    dec[:, 1::2] = oracle.e2m1_decode(P.bb.codes >> 4)
+    sc = (oracle.e4m3_decode(P.bb.scales) if fmt == "nvfp4"
+          else oracle.e8m0_decode(P.bb.scales))
+    Db = (dec * np.repeat(sc, blk, axis=1)).astype(np.float32) * np.float32(P.bb.tscale)
+    assert np.array_equal((Db + P.r).astype(np.float32), P.y)
+    # pruned positions carry code 0 and their residual is y itself
+    keep = np.unpackbits(P.mask, axis=1, bitorder="little").astype(bool)
+    assert np.all(np.where(keep, True, (dec == 0) & ~np.signbit(dec)))
+    assert np.array_equal(P.r[~keep], P.y[~keep])
+    assert np.all(keep.reshape(6, -1, m).sum(axis=2) == n)
+    # the residual is not the unquantised complement: kept entries differ
+    assert np.any(P.r[keep] != 0)
+
+
+def test_prepare_on_grid_sparse_input_has_zero_residual():
+    """Input already on the NVFP4 grid with <= n nonzeros per group: the
+    backbone holds it exactly, so the residual is zero (tensor scale 1)."""
+    rng = np.random.default_rng(13)
+    T = _grid_tensor_nvfp4(rng, 4, 256, 0, sparse24=True)
+    X = _bf16(T)
+    assert np.array_equal(wl.bf16_bits_to_f32(X), T)
+    P = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4")
+    assert np.all(P.rs.codes == 0) and P.rs.tscale == 1.0
+    assert P.bb.tscale == 1.0
+
+
+def test_prepare_commutes_with_row_gather():
+    X = wl.activation("laplace_outlier", 14, 0, 9, 512)
+    P = oracle.prepare(X, wl.gamma_ones(512), 1e-6)
+    idx = np.array([3, 3, 0, 8, 1, 1, 1, 5, 2, 4, 6, 7])
+    Q = oracle.prepare(X[idx], wl.gamma_ones(512), 1e-6)
+    assert Q.bb.tscale == P.bb.tscale and Q.rs.tscale == P.rs.tscale
+    for a, b in [(Q.bb.codes, P.bb.codes), (Q.bb.scales, P.bb.scales),
+                 (Q.rs.codes, P.rs.codes), (Q.rs.scales, P.rs.scales), (Q.mask, P.mask)]:
+        assert np.array_equal(a, b[idx])
+
+
+# ---------------------------------------------------------------- GEMM -----
+
+def test_linear_bruteforce_tiny():
+    X = wl.activation("normal_outlier", 1, 0, 3, 64)
+    W = wl.weight(1, 0, 5, 64)
+    P = oracle.prepare(X, wl.gamma_ones(64), 1e-6)
+    Wq = oracle.quantize_weight(W)
+    Y = oracle.linear(P, Wq)
+
+    def val(codes, scales, i, k):
+        byte = int(codes[i, k // 2])
+        c = byte & 15 if k % 2 == 0 else byte >> 4
+        mag = [0, .5, 1, 1.5, 2, 3, 4, 6][c & 7] * (-1 if c & 8 else 1)
+        return mag * float(oracle.e4m3_decode(np.array([scales[i, k // 16]]))[0])
+
+    for i in range(3):
+        for j in range(5):
+            sb = sr = 0.0
+            for k in range(64):
+                w = val(Wq.codes, Wq.scales, j, k)
+                sb += val(P.bb.codes, P.bb.scales, i, k) * w
+                sr += val(P.rs.codes, P.rs.scales, i, k) * w
+            want = float(Wq.tscale) * (float(P.bb.tscale) * sb + float(P.rs.tscale) * sr)
+            assert abs(Y[i, j] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_linear_on_grid_equals_plain_matmul():
+    """X on the grid with r = 0 and W on the grid: the two-path linear is the
+    plain fp64 product of the original values."""
+    rng = np.random.default_rng(15)
+    T = _grid_tensor_nvfp4(rng, 6, 256, -4, sparse24=True)
+    W = _grid_tensor_nvfp4(rng, 16, 256, -9)
+    P = oracle.prepare(_bf16(T), None, 1e-6, 2, 4, "nvfp4")
+    Wq = oracle.quantize_weight(_bf16(W))
+    Y = oracle.linear(P, Wq)
+    ref = T.astype(np.float64) @ W.astype(np.float64).T
+    assert np.allclose(Y, ref, rtol=1e-13, atol=1e-13 * np.abs(ref).max())
+
+
+def test_linear_dense_residual_compensates():
+    """The two-path result is closer to the unquantised product than the
+    backbone path alone (the residual path carries mask loss and backbone
+    quantisation error)."""
+    X = wl.activation("laplace_outlier", 16, 0, 32, 1024)
+    W = wl.weight(16, 0, 64, 1024)
+    P = oracle.prepare(X, wl.gamma_ones(1024), 1e-6, keep_intermediates=True)
+    Wq = oracle.quantize_weight(W)
+    Y = oracle.linear(P, Wq)
+    Dw = oracle.dequant_blocks(Wq) * float(Wq.tscale)
+    exact = P.y.astype(np.float64) @ Dw.T
+    bb_only = float(Wq.tscale) * float(P.bb.tscale) * (oracle.dequant_blocks(P.bb) @ oracle.dequant_blocks(Wq).T)
+    assert np.linalg.norm(Y - exact) < 0.5 * np.linalg.norm(bb_only - exact)
+
+
+def test_bf16_rne_reference():
+    v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -(1.0 + 2 ** -8), 1e-40, 3.0e38,
+                  1.00390625 + 1e-12], dtype=np.float64)
+    got = wl.bf16_bits_to_f32(oracle.bf16_rne_from_f64(v)).astype(np.float64)
+    want = [1.0, 1.0, 1.0 + 2 ** -7, -1.0, None, None, 1.0078125]
+    assert got[0] == want[0] and got[1] == want[1] and got[2] == want[2] and got[3] == want[3]
+    assert got[6] == want[6]
+
+
+def test_moe_reduces_to_per_expert_linear():
+    X = wl.activation("laplace_outlier", 17, 0, 10, 256)
+    P = oracle.prepare(X, wl.gamma_ones(256), 1e-6)
+    experts = [oracle.quantize_weight(wl.weight(17, e, 32, 256)) for e in range(3)]
+    ex = np.array([[0, 2], [1, 2], [0, 1], [2, 0], [1, 0], [0, 2], [2, 1], [0, 1], [1, 2], [2, 0]])
+    ri, off = wl.group_by_expert(ex.astype(np.int32), 3)
+    Y = oracle.moe_linear(P, ri, off, experts)
+    for t in range(len(ri)):
+        e = int(np.searchsorted(off, t, side="right") - 1)
+        want = oracle.linear(oracle.gather_rows(P, ri[t:t + 1]), experts[e])[0]
+        assert np.array_equal(Y[t], want)
