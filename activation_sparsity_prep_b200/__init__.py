@@ -1,0 +1,255 @@
+"""SharQ hot path on B200 (sm_100a): Python binding of libsharq.
+
+Thin ctypes marshalling over the C ABI declared in ``include/sharq.h``.
+PyTorch supplies device memory and the current CUDA stream; every step of
+the computation runs in the library's CUDA kernels.  There is no CPU
+fallback: without the compiled library every call raises.
+
+SharQ paper, Abstract: a fused preparation operator (normalisation, an
+input-adaptive N:M mask, an FP4 backbone and an FP4 residual taken against
+the dequantised backbone) feeds a sparse FP4 GEMM and a dense FP4 GEMM that
+share one FP4 weight payload.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional
+
+__all__ = [
+    "NVFP4", "MXFP4", "SharqError", "load_sharq_ops", "scale_bytes",
+    "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
+    "prepare", "linear", "moe_linear", "last_device_status",
+]
+
+NVFP4, MXFP4 = 0, 1
+_FMT = {"nvfp4": NVFP4, "mxfp4": MXFP4}
+_BLOCK = {NVFP4: 16, MXFP4: 32}
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration",
+           3: "CUDA error", 4: "device wait timed out"}
+
+
+class SharqError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("N", ctypes.c_int),
+                ("K", ctypes.c_int), ("fmt", ctypes.c_int)]
+
+
+class _Prepared(ctypes.Structure):
+    _fields_ = [("bb_codes", ctypes.c_void_p), ("bb_scales", ctypes.c_void_p),
+                ("bb_tscale", ctypes.c_void_p), ("rs_codes", ctypes.c_void_p),
+                ("rs_scales", ctypes.c_void_p), ("rs_tscale", ctypes.c_void_p),
+                ("mask", ctypes.c_void_p), ("M", ctypes.c_int), ("K", ctypes.c_int),
+                ("n", ctypes.c_int), ("m", ctypes.c_int), ("fmt", ctypes.c_int)]
+
+
+_lib = None
+_lock = threading.Lock()
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsharq.so")
+
+
+def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libsharq.so (building it with nvcc when it is missing or older
+    than its sources).  Raises if the library cannot be produced."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if build_if_missing:
+            from . import build as _build
+            if not _build.up_to_date():
+                _build.build()
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libsharq.so not found at {LIB_PATH}; run "
+                              "python -m activation_sparsity_prep_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.sharq_status_string.argtypes = [I]
+        L.sharq_status_string.restype = ctypes.c_char_p
+        L.sharq_scale_bytes.argtypes = [I64, I, I]
+        L.sharq_scale_bytes.restype = SZ
+        L.sharq_prepare_workspace_bytes.argtypes = [I64, I, I]
+        L.sharq_prepare_workspace_bytes.restype = SZ
+        L.sharq_quantize_weight.argtypes = [P, ctypes.POINTER(_Weight), P, SZ, P]
+        L.sharq_quantize_weight.restype = I
+        L.sharq_prepare.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P, SZ, P]
+        L.sharq_prepare.restype = I
+        L.sharq_linear.argtypes = [ctypes.POINTER(_Prepared), ctypes.POINTER(_Weight), P, I, P]
+        L.sharq_linear.restype = I
+        L.sharq_moe_linear.argtypes = [ctypes.POINTER(_Prepared), P, P, I, I64,
+                                       ctypes.POINTER(_Weight), P, I, P]
+        L.sharq_moe_linear.restype = I
+        L.sharq_last_device_status.argtypes = [P]
+        L.sharq_last_device_status.restype = I
+        _lib = L
+        return L
+
+
+def _fmt(fmt) -> int:
+    return _FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise SharqError(fn, st)
+
+
+def scale_bytes(rows: int, K: int, fmt="nvfp4") -> int:
+    return int(load_sharq_ops().sharq_scale_bytes(rows, K, _fmt(fmt)))
+
+
+def prepare_workspace_bytes(M: int, K: int, fmt="nvfp4") -> int:
+    return int(load_sharq_ops().sharq_prepare_workspace_bytes(M, K, _fmt(fmt)))
+
+
+@dataclass
+class Weight:
+    """Shared FP4 weight payload (device tensors)."""
+    codes: "object"          # uint8 [N, K/2] (or [E, N, K/2])
+    scales: "object"         # uint8 MMA-ready atoms
+    tensor_scale: "object"   # fp32 [1] (or [E])
+    N: int
+    K: int
+    fmt: int
+    E: int = 1
+
+    def _c(self) -> _Weight:
+        return _Weight(_ptr(self.codes), _ptr(self.scales), _ptr(self.tensor_scale),
+                       self.N, self.K, self.fmt)
+
+    @staticmethod
+    def empty(N: int, K: int, fmt="nvfp4", device="cuda", E: int = 1) -> "Weight":
+        import torch
+        f = _fmt(fmt)
+        sb = scale_bytes(N, K, f)
+        shape = (N, K // 2) if E == 1 else (E, N, K // 2)
+        return Weight(torch.empty(shape, dtype=torch.uint8, device=device),
+                      torch.empty((E * sb,), dtype=torch.uint8, device=device),
+                      torch.empty((E,), dtype=torch.float32, device=device), N, K, f, E)
+
+
+@dataclass
+class Prepared:
+    """Backbone and residual FP4 operands produced by prepare()."""
+    bb_codes: "object"
+    bb_scales: "object"
+    bb_tscale: "object"
+    rs_codes: "object"
+    rs_scales: "object"
+    rs_tscale: "object"
+    mask: "object"
+    M: int
+    K: int
+    n: int
+    m: int
+    fmt: int
+
+    def _c(self) -> _Prepared:
+        return _Prepared(_ptr(self.bb_codes), _ptr(self.bb_scales), _ptr(self.bb_tscale),
+                         _ptr(self.rs_codes), _ptr(self.rs_scales), _ptr(self.rs_tscale),
+                         _ptr(self.mask), self.M, self.K, self.n, self.m, self.fmt)
+
+    @staticmethod
+    def empty(M: int, K: int, n: int = 2, m: int = 4, fmt="nvfp4", want_mask: bool = False,
+              device="cuda") -> "Prepared":
+        import torch
+        f = _fmt(fmt)
+        sb = scale_bytes(M, K, f)
+        u8 = dict(dtype=torch.uint8, device=device)
+        return Prepared(torch.empty((M, K // 2), **u8), torch.empty((sb,), **u8),
+                        torch.empty((1,), dtype=torch.float32, device=device),
+                        torch.empty((M, K // 2), **u8), torch.empty((sb,), **u8),
+                        torch.empty((1,), dtype=torch.float32, device=device),
+                        torch.empty((M, K // 8), **u8) if want_mask else None,
+                        M, K, n, m, f)
+
+
+def _workspace(M: int, K: int, fmt: int, ws=None, device="cuda"):
+    import torch
+    need = prepare_workspace_bytes(M, K, fmt)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=device)
+    return ws
+
+
+def quantize_weight(W, fmt="nvfp4", out: Optional[Weight] = None, ws=None, stream=None) -> Weight:
+    """W: bf16 [N, K] device tensor -> shared FP4 payload."""
+    L = load_sharq_ops()
+    N, K = W.shape
+    f = _fmt(fmt)
+    w = out if out is not None else Weight.empty(N, K, f, device=W.device)
+    ws = _workspace(N, K, f, ws, W.device)
+    cw = w._c()
+    _check("sharq_quantize_weight",
+           L.sharq_quantize_weight(W.data_ptr(), ctypes.byref(cw), ws.data_ptr(), ws.numel(),
+                                   _stream(stream)))
+    return w
+
+
+def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4",
+            want_mask: bool = False, out: Optional[Prepared] = None, ws=None,
+            stream=None) -> Prepared:
+    """X: bf16 [M, K] device tensor; gamma: bf16 [K] or None (no norm)."""
+    L = load_sharq_ops()
+    M, K = X.shape
+    f = _fmt(fmt)
+    p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device)
+    ws = _workspace(M, K, f, ws, X.device)
+    cp = p._c()
+    _check("sharq_prepare",
+           L.sharq_prepare(X.data_ptr(), _ptr(gamma), float(eps), ctypes.byref(cp),
+                           ws.data_ptr(), ws.numel(), _stream(stream)))
+    return p
+
+
+def linear(x: Prepared, w: Weight, out_fp32: bool = False, out=None, stream=None):
+    """Two-path FP4 linear: Y = G_w (G_b A_b W^T + G_r A_r W^T)."""
+    import torch
+    L = load_sharq_ops()
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    Y = out if out is not None else torch.empty((x.M, w.N), dtype=dt, device=x.bb_codes.device)
+    cx, cw = x._c(), w._c()
+    _check("sharq_linear", L.sharq_linear(ctypes.byref(cx), ctypes.byref(cw), Y.data_ptr(),
+                                          1 if out_fp32 else 0, _stream(stream)))
+    return Y
+
+
+def moe_linear(x: Prepared, row_index, offsets, w: Weight, out_fp32: bool = False, out=None,
+               stream=None):
+    """Grouped two-path linear; row_index: int32 [T] device tensor or None,
+    offsets: int32 [E+1] device tensor, w: stacked expert weights."""
+    import torch
+    L = load_sharq_ops()
+    T = int(row_index.numel()) if row_index is not None else x.M
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    Y = out if out is not None else torch.empty((T, w.N), dtype=dt, device=x.bb_codes.device)
+    cx, cw = x._c(), w._c()
+    _check("sharq_moe_linear",
+           L.sharq_moe_linear(ctypes.byref(cx), _ptr(row_index), offsets.data_ptr(),
+                              int(offsets.numel()) - 1, T, ctypes.byref(cw), Y.data_ptr(),
+                              1 if out_fp32 else 0, _stream(stream)))
+    return Y
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise and return (then clear) the device status word."""
+    return int(load_sharq_ops().sharq_last_device_status(_stream(stream)))

@@ -1,0 +1,168 @@
+// abi.cu -- extern "C" entry points of libsharq (declared in include/sharq.h).
+//
+// Argument validation happens here, on the host, before anything is
+// enqueued; the kernels themselves live in prepare.cu and linear.cu.
+#include "../../include/sharq.h"
+#include "common.cuh"
+#include "sharq_internal.h"
+
+#include <mutex>
+
+namespace sharq {
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static std::mutex mu;
+    static int cache[64] = {0};
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+}  // namespace sharq
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_fmt(int fmt) { return fmt == SHARQ_NVFP4 || fmt == SHARQ_MXFP4; }
+
+bool valid_shape(int64_t rows, int K) { return rows >= 0 && K > 0 && K % 256 == 0; }
+
+sharq_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return SHARQ_OK;
+    if (e == cudaErrorNotSupported) return SHARQ_ERR_UNSUPPORTED;
+    return SHARQ_ERR_CUDA;
+}
+
+int block_size(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
+
+}  // namespace
+
+extern "C" {
+
+const char* sharq_status_string(int status) {
+    switch (status) {
+        case SHARQ_OK: return "ok";
+        case SHARQ_ERR_INVALID_ARG: return "invalid argument";
+        case SHARQ_ERR_UNSUPPORTED: return "unsupported configuration";
+        case SHARQ_ERR_CUDA: return "CUDA error";
+        case SHARQ_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+size_t sharq_scale_bytes(int64_t rows, int K, int fmt) {
+    if (!valid_fmt(fmt) || !valid_shape(rows, K)) return 0;
+    int64_t rpad = (rows + 127) / 128 * 128;
+    return (size_t)(rpad * (K / block_size(fmt)));
+}
+
+size_t sharq_prepare_workspace_bytes(int64_t M, int K, int fmt) {
+    if (!valid_fmt(fmt) || !valid_shape(M, K)) return 0;
+    return sharq::prepare_ws_bytes(M);
+}
+
+sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_weight* out, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    if (!out || !W_bf16 || !ws) return SHARQ_ERR_INVALID_ARG;
+    if (!valid_fmt(out->fmt) || !valid_shape(out->N, out->K) || out->N % 128 != 0 || out->N == 0)
+        return SHARQ_ERR_INVALID_ARG;
+    if (!out->codes || !out->scales || !out->tensor_scale) return SHARQ_ERR_INVALID_ARG;
+    if (!aligned16(W_bf16) || !aligned16(out->codes) || !aligned16(out->scales) || !aligned16(ws) ||
+        ((uintptr_t)out->tensor_scale & 3u))
+        return SHARQ_ERR_INVALID_ARG;
+    if (ws_bytes < sharq::prepare_ws_bytes(out->N)) return SHARQ_ERR_INVALID_ARG;
+    sharq::PrepareLaunch p{};
+    p.X = W_bf16; p.gamma = nullptr; p.eps = 0.f; p.M = out->N; p.K = out->K;
+    p.n = 8; p.m = 8; p.fmt = out->fmt; p.weight = true;
+    p.bb_codes = out->codes; p.bb_scales = out->scales; p.bb_tscale = out->tensor_scale;
+    p.ws = ws;
+    return cuda_status(sharq::launch_prepare(p, static_cast<cudaStream_t>(stream),
+                                             sharq::device_sm_count()));
+}
+
+sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps,
+                           const sharq_prepared* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!out || !ws) return SHARQ_ERR_INVALID_ARG;
+    const sharq_prepared& o = *out;
+    if (!valid_fmt(o.fmt) || !valid_shape(o.M, o.K)) return SHARQ_ERR_INVALID_ARG;
+    if (!(o.m == 2 || o.m == 4 || o.m == 8) || o.n < 1 || o.n > o.m) return SHARQ_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !(eps < 1e30f)) return SHARQ_ERR_INVALID_ARG;
+    if ((o.M > 0 && !X_bf16) || !o.bb_codes || !o.bb_scales || !o.bb_tscale || !o.rs_codes ||
+        !o.rs_scales || !o.rs_tscale)
+        return SHARQ_ERR_INVALID_ARG;
+    if (!aligned16(X_bf16) || !aligned16(gamma_bf16) || !aligned16(o.bb_codes) ||
+        !aligned16(o.bb_scales) || !aligned16(o.rs_codes) || !aligned16(o.rs_scales) ||
+        !aligned16(o.mask) || !aligned16(ws) || ((uintptr_t)o.bb_tscale & 3u) ||
+        ((uintptr_t)o.rs_tscale & 3u))
+        return SHARQ_ERR_INVALID_ARG;
+    if (ws_bytes < sharq::prepare_ws_bytes(o.M)) return SHARQ_ERR_INVALID_ARG;
+    sharq::PrepareLaunch p{};
+    p.X = X_bf16; p.gamma = gamma_bf16; p.eps = eps; p.M = o.M; p.K = o.K; p.n = o.n; p.m = o.m;
+    p.fmt = o.fmt; p.weight = false;
+    p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
+    p.rs_codes = o.rs_codes; p.rs_scales = o.rs_scales; p.rs_tscale = o.rs_tscale;
+    p.mask = o.mask; p.ws = ws;
+    return cuda_status(sharq::launch_prepare(p, static_cast<cudaStream_t>(stream),
+                                             sharq::device_sm_count()));
+}
+
+static sharq_status check_linear_args(const sharq_prepared* x, const sharq_weight* w, void* Y) {
+    if (!x || !w || !Y) return SHARQ_ERR_INVALID_ARG;
+    if (!valid_fmt(x->fmt) || x->fmt != w->fmt) return SHARQ_ERR_INVALID_ARG;
+    if (!valid_shape(x->M, x->K) || x->K != w->K) return SHARQ_ERR_INVALID_ARG;
+    if (w->N <= 0 || w->N % 128 != 0) return SHARQ_ERR_INVALID_ARG;
+    if (!x->bb_codes || !x->bb_scales || !x->bb_tscale || !x->rs_codes || !x->rs_scales ||
+        !x->rs_tscale || !w->codes || !w->scales || !w->tensor_scale)
+        return SHARQ_ERR_INVALID_ARG;
+    if (!aligned16(x->bb_codes) || !aligned16(x->bb_scales) || !aligned16(x->rs_codes) ||
+        !aligned16(x->rs_scales) || !aligned16(w->codes) || !aligned16(w->scales) || !aligned16(Y))
+        return SHARQ_ERR_INVALID_ARG;
+    return SHARQ_OK;
+}
+
+sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w, void* Y, int y_is_fp32,
+                          void* stream) {
+    sharq_status st = check_linear_args(x, w, Y);
+    if (st != SHARQ_OK) return st;
+    sharq::LinearLaunch p{};
+    p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
+    p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
+    p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
+    p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
+    return cuda_status(sharq::launch_linear(p, static_cast<cudaStream_t>(stream),
+                                            sharq::device_sm_count()));
+}
+
+sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
+                              const int32_t* expert_offsets, int E, int64_t T,
+                              const sharq_weight* w, void* Y, int y_is_fp32, void* stream) {
+    sharq_status st = check_linear_args(x, w, Y);
+    if (st != SHARQ_OK) return st;
+    if (!expert_offsets || E <= 0 || T < 0 || (!row_index && T != x->M)) return SHARQ_ERR_INVALID_ARG;
+    sharq::LinearLaunch p{};
+    p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
+    p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
+    p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
+    p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
+    p.row_index = row_index; p.offsets = expert_offsets; p.E = E; p.T = T;
+    return cuda_status(sharq::launch_moe_linear(p, static_cast<cudaStream_t>(stream),
+                                                sharq::device_sm_count()));
+}
+
+sharq_status sharq_last_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return SHARQ_ERR_CUDA;
+    unsigned v = sharq::take_status_prepare() | sharq::take_status_linear();
+    if (v & sharq::kStatusReadFailed) return SHARQ_ERR_CUDA;
+    if (v & (sharq::kStatusGridTimeout | sharq::kStatusMbarTimeout)) return SHARQ_ERR_TIMEOUT;
+    if (v) return SHARQ_ERR_CUDA;
+    return SHARQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// sharq_internal.h -- host-side launch interfaces between the C ABI layer
+// and the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace sharq {
+
+struct PrepareLaunch {
+    const void* X;
+    const void* gamma;
+    float eps;
+    int64_t M;
+    int K, n, m, fmt;
+    bool weight;          // quantise a whole weight tensor (keep-all, no residual)
+    void* bb_codes;
+    void* bb_scales;
+    float* bb_tscale;
+    void* rs_codes;
+    void* rs_scales;
+    float* rs_tscale;
+    void* mask;
+    void* ws;
+};
+
+size_t prepare_ws_bytes(int64_t M);
+cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms);
+
+struct LinearLaunch {
+    const void* bb_codes;
+    const void* bb_scales;
+    const float* bb_tscale;
+    const void* rs_codes;
+    const void* rs_scales;
+    const float* rs_tscale;
+    const void* w_codes;      // expert 0 for the grouped form
+    const void* w_scales;
+    const float* w_tscale;
+    int64_t M;                // rows of the prepared operands
+    int N, K, fmt;
+    void* Y;
+    int y_fp32;
+    // grouped form
+    const int32_t* row_index; // may be null
+    const int32_t* offsets;   // null for the plain linear
+    int E;
+    int64_t T;
+};
+
+cudaError_t launch_linear(const LinearLaunch& p, cudaStream_t s, int sms);
+cudaError_t launch_moe_linear(const LinearLaunch& p, cudaStream_t s, int sms);
+
+int device_sm_count();
+
+// Read and clear the device status words of each kernel file.
+unsigned take_status_prepare();
+unsigned take_status_linear();
+
+}  // namespace sharq

@@ -1,0 +1,168 @@
+/*
+ * sharq.h -- C ABI of the B200 (sm_100a) SharQ hot path.
+ *
+ * SharQ (SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
+ * Inference, arXiv 2606.26587, Abstract) splits each linear layer's input
+ * online into an outlier-dominated N:M-sparse backbone and a dense residual
+ * taken against the *dequantised* backbone, quantises both to FP4, and runs
+ * a sparse FP4 GEMM on the backbone plus a dense FP4 GEMM on the residual,
+ * both reading one shared FP4 weight payload with per-path scale views.  A
+ * fused preparation operator absorbs normalisation, mask generation and
+ * residual construction.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library allocates nothing and keeps no reference after a call returns.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Work is enqueued asynchronously; no call synchronises except
+ *     sharq_last_device_status().
+ *   - Pointers must be 16-byte aligned.  K % 256 == 0, N % 128 == 0, M >= 0.
+ *   - A violated precondition returns SHARQ_ERR_INVALID_ARG (or
+ *     SHARQ_ERR_UNSUPPORTED for a valid but unimplemented choice) before any
+ *     work is enqueued.  A failed launch returns SHARQ_ERR_CUDA.  A bounded
+ *     device-side wait that gives up (about one second) records a timeout in
+ *     a device status word that sharq_last_device_status() reports.
+ *   - Inputs must be finite.  Non-finite inputs are outside the contract.
+ *
+ * Data layouts (all row-major unless stated)
+ *   bf16 tensors           raw bfloat16, [rows, K]
+ *   FP4 codes              uint8 [rows, K/2]; E2M1 element 2j in bits 3:0 and
+ *                          element 2j+1 in bits 7:4 of byte j
+ *   block scales           "MMA-ready" atoms: rows are padded to a multiple
+ *                          of 128 and the scale matrix [rows_pad, K/B] (B =
+ *                          16 for NVFP4 with E4M3 codes, 32 for MXFP4 with
+ *                          E8M0 codes) is stored as 512-byte atoms of 128 rows
+ *                          x 4 scales.  Scale (r, s) lives at byte
+ *                            ((r/128) * (K/B/4) + s/4) * 512
+ *                            + (r%32) * 16 + ((r%128)/32) * 4 + s%4.
+ *                          sharq_scale_bytes() gives the buffer size.
+ *   tensor scale           one fp32 decode scale G (NVFP4: amax / 2688; it
+ *                          is 1.0 for MXFP4 and for an all-zero tensor)
+ *   mask (optional)        uint8 [M, K/8]; bit t of byte j set when element
+ *                          8j+t is in the backbone
+ */
+#ifndef SHARQ_H
+#define SHARQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SHARQ_API __attribute__((visibility("default")))
+#else
+#define SHARQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SHARQ_OK = 0,
+    SHARQ_ERR_INVALID_ARG = 1,
+    SHARQ_ERR_UNSUPPORTED = 2,
+    SHARQ_ERR_CUDA = 3,
+    SHARQ_ERR_TIMEOUT = 4
+} sharq_status;
+
+typedef enum {
+    SHARQ_NVFP4 = 0,   /* E2M1 codes, E4M3 scale per 16 elements, fp32 tensor scale */
+    SHARQ_MXFP4 = 1    /* E2M1 codes, E8M0 scale per 32 elements, no tensor scale   */
+} sharq_format;
+
+/* One FP4 weight payload shared by both GEMM paths (Abstract: a single FP4
+ * weight payload with path-specific scale views).  Both paths use the same
+ * codes and the same MMA-ready scale atoms, which is the layout the block-
+ * scaled MMA reads for either path, so one scale copy serves as both views.
+ * For a stacked (grouped) weight: codes [E, N, K/2], scales E consecutive
+ * buffers of sharq_scale_bytes(N, K, fmt) bytes, tensor_scale [E]. */
+typedef struct {
+    void*  codes;
+    void*  scales;
+    float* tensor_scale;
+    int    N, K;
+    int    fmt;          /* sharq_format */
+} sharq_weight;
+
+/* Output of the preparation operator: the backbone and residual operands. */
+typedef struct {
+    void*  bb_codes;     /* [M, K/2]                                        */
+    void*  bb_scales;    /* sharq_scale_bytes(M, K, fmt) bytes              */
+    float* bb_tscale;    /* [1] backbone decode scale G_b                   */
+    void*  rs_codes;     /* [M, K/2]                                        */
+    void*  rs_scales;    /* sharq_scale_bytes(M, K, fmt) bytes              */
+    float* rs_tscale;    /* [1] residual decode scale G_r                   */
+    void*  mask;         /* optional [M, K/8] bitmask, NULL to skip         */
+    int    M, K, n, m;
+    int    fmt;          /* sharq_format */
+} sharq_prepared;
+
+/* Human-readable name of a status code (static string). */
+SHARQ_API const char* sharq_status_string(int status);
+
+/* Bytes of one MMA-ready block-scale buffer for `rows` x K (rows padded to
+ * 128).  Returns 0 for invalid arguments. */
+SHARQ_API size_t sharq_scale_bytes(int64_t rows, int K, int fmt);
+
+/* Workspace the preparation operator needs (tensor-wide maxima, a grid
+ * barrier and one fp32 per row).  Caller-owned device memory; its content on
+ * entry does not matter.  Calls that share a workspace must not overlap. */
+SHARQ_API size_t sharq_prepare_workspace_bytes(int64_t M, int K, int fmt);
+
+/* Offline weight quantisation (once per layer; Abstract: shared FP4 weight
+ * payload).  W bf16 [N, K] -> out->codes, out->scales, out->tensor_scale,
+ * with NVFP4 scales from the tensor-wide amax (G = amax / 2688, block scale
+ * E4M3(amax_block * 2688 / (6 * amax))) or MXFP4 scales (E8M0 exponent
+ * floor(log2 amax_block) - 2).  `out->N, K, fmt` must be filled in by the
+ * caller.  ws: sharq_prepare_workspace_bytes(N, K, fmt) bytes. */
+SHARQ_API sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_weight* out,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Fused preparation operator (Abstract: one operator absorbing layer
+ * normalisation, mask generation and residual construction).  For X bf16
+ * [M, K]:
+ *   y   = RMSNorm(X) * gamma per row (fp32, fixed reduction order), or y = X
+ *         when gamma is NULL;
+ *   keep: in every aligned group of m along K the n entries of largest |y|
+ *         (lower index first on ties);
+ *   backbone B = keep ? y : 0, quantised to FP4 with its own tensor scale;
+ *   residual r = y - dequant(Q(B)), quantised to FP4 with its own tensor
+ *         scale.
+ * Fills the buffers named in *out (out->M, K, n, m, fmt must match the
+ * arguments).  Supported: m in {2, 4, 8}, 1 <= n <= m.  ws:
+ * sharq_prepare_workspace_bytes(M, K, fmt) bytes. */
+SHARQ_API sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps,
+                           const sharq_prepared* out, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Two-path FP4 linear (Abstract: a sparse FP4 GEMM on the backbone and a
+ * dense FP4 GEMM on the residual, one shared weight payload):
+ *   Y[i,j] = G_w * (G_b * S_b[i,j] + G_r * S_r[i,j]),
+ *   S_p = sum_k val(p)[i,k] s(p)[i,k/B] * val(w)[j,k] s(w)[j,k/B].
+ * Both products accumulate in fp32 tensor memory from one weight tile per
+ * k-step.  Y is bf16 [M, N] (y_is_fp32 = 0) or fp32 [M, N]. */
+SHARQ_API sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w,
+                          void* Y, int y_is_fp32, void* stream);
+
+/* Grouped (mixture-of-experts) form of sharq_linear: dispatched row t
+ * (0 <= t < T) reads prepared row row_index[t] (row_index NULL: row t) and is
+ * multiplied by expert e's weight when offsets[e] <= t < offsets[e+1].
+ * expert_offsets is a DEVICE int32 array [E+1] with offsets[0] = 0 and
+ * offsets[E] = T, non-decreasing.  w holds E stacked weights (see
+ * sharq_weight).  The activation tensor scales are those of the whole
+ * prepare call.  Y is [T, N]. */
+SHARQ_API sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
+                              const int32_t* expert_offsets, int E, int64_t T,
+                              const sharq_weight* w, void* Y, int y_is_fp32,
+                              void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word:
+ * SHARQ_OK, SHARQ_ERR_TIMEOUT if a bounded device wait gave up since the
+ * last call, or SHARQ_ERR_CUDA if the stream itself reports an error. */
+SHARQ_API sharq_status sharq_last_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHARQ_H */

@@ -1,0 +1,83 @@
+"""CPU-side checks of the C ABI: the library builds and loads, exports every
+symbol include/sharq.h declares, and rejects bad arguments on the host
+before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import activation_sparsity_prep_b200 as sq
+from tests.sharq_testlib import atom_index
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "sharq.h")).read()
+    return re.findall(r"SHARQ_API\s+[\w\s\*]+?\b(sharq_\w+)\s*\(", src)
+
+
+def test_library_exports_every_declared_symbol():
+    L = sq.load_sharq_ops()
+    names = _declared()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_scale_and_workspace_sizes():
+    assert sq.scale_bytes(16, 256, "nvfp4") == 128 * 16
+    assert sq.scale_bytes(129, 4096, "nvfp4") == 256 * 256
+    assert sq.scale_bytes(128, 4096, "mxfp4") == 128 * 128
+    assert sq.scale_bytes(16, 100, "nvfp4") == 0          # K % 256 != 0
+    assert sq.prepare_workspace_bytes(1000, 4096) >= 64 + 4 * 1000
+    assert sq.scale_bytes(0, 256) == 0
+
+
+def test_atom_layout_is_a_permutation():
+    idx = atom_index(256, 1024, "nvfp4")
+    assert np.array_equal(np.sort(idx.ravel()), np.arange(256 * 64))
+
+
+def _fake_prepared(M=16, K=256, n=2, m=4, fmt=0, p=0x1000):
+    return sq._Prepared(p, p, p, p, p, p, None, M, K, n, m, fmt)
+
+
+@pytest.mark.parametrize("kw", [dict(K=100), dict(m=3), dict(n=0), dict(n=5), dict(fmt=7),
+                                dict(M=-1), dict(p=0x1001)])
+def test_prepare_rejects_bad_arguments_on_host(kw):
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared(**kw)
+    st = L.sharq_prepare(0x1000, None, 1e-6, ctypes.byref(cp), 0x1000, 1 << 20, None)
+    assert st == 1
+
+
+def test_prepare_rejects_small_workspace_and_bad_eps():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    assert L.sharq_prepare(0x1000, None, 1e-6, ctypes.byref(cp), 0x1000, 8, None) == 1
+    assert L.sharq_prepare(0x1000, None, float("nan"), ctypes.byref(cp), 0x1000, 1 << 20, None) == 1
+    assert L.sharq_prepare(0x1000, None, 1e-6, None, 0x1000, 1 << 20, None) == 1
+
+
+def test_linear_rejects_mismatched_operands():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 512, 0)          # K mismatch
+    assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0, None) == 1
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 200, 256, 0)          # N % 128
+    assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0, None) == 1
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 1)          # format mismatch
+    assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0, None) == 1
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 0)
+    assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1008, 0, None) == 1   # misaligned Y
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, None, 4, 16, ctypes.byref(w), 0x1000, 0, None) == 1
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 4, 17, ctypes.byref(w), 0x1000, 0, None) == 1
+
+
+def test_status_strings():
+    L = sq.load_sharq_ops()
+    assert L.sharq_status_string(0) == b"ok"
+    assert L.sharq_status_string(4) == b"device wait timed out"

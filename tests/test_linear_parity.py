@@ -1,0 +1,139 @@
+"""GPU parity of the two-path tcgen05 FP4 linear against the fp64 oracle.
+
+Tolerances (from the stated target): the fp32 output within a relative
+Frobenius error of 1e-5 of the fp64 reference, and the bf16 output within
+one bf16 ulp of the correctly rounded fp64 result, element by element."""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparsity_prep_b200 as sq
+from activation_sparsity_prep_b200 import workloads as wl
+import oracle
+from tests.sharq_testlib import canonical_to_atoms, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+FROB_TOL = 1e-5
+
+
+def bf16_ordered(b):
+    b = b.astype(np.int64)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def upload_prepared(R, M, K, fmt):
+    """Oracle operands -> device buffers in the library's layouts."""
+    f = sq._FMT[fmt]
+    P = sq.Prepared.empty(M, K, R.n, R.m, f)
+    P.bb_codes.copy_(torch.from_numpy(R.bb.codes))
+    P.rs_codes.copy_(torch.from_numpy(R.rs.codes))
+    P.bb_scales.copy_(torch.from_numpy(canonical_to_atoms(R.bb.scales, K, fmt)))
+    P.rs_scales.copy_(torch.from_numpy(canonical_to_atoms(R.rs.scales, K, fmt)))
+    P.bb_tscale.fill_(float(R.bb.tscale))
+    P.rs_tscale.fill_(float(R.rs.tscale))
+    return P
+
+
+def upload_weight(Rw, N, K, fmt):
+    w = sq.Weight.empty(N, K, fmt)
+    w.codes.copy_(torch.from_numpy(Rw.codes))
+    w.scales.copy_(torch.from_numpy(canonical_to_atoms(Rw.scales, K, fmt)))
+    w.tensor_scale.fill_(float(Rw.tscale))
+    return w
+
+
+def check(Y32, Ybf, Y64, rows=None):
+    Y32 = to_np(Y32).astype(np.float64)
+    if rows is not None:
+        Y32 = Y32[rows]
+    err = np.linalg.norm(Y32 - Y64) / max(np.linalg.norm(Y64), 1e-300)
+    assert err <= FROB_TOL, f"relative Frobenius error {err:.3e}"
+    ref = oracle.bf16_rne_from_f64(Y64)
+    got = to_np(Ybf)
+    if rows is not None:
+        got = got[rows]
+    d = np.abs(bf16_ordered(got) - bf16_ordered(ref))
+    assert d.max() <= 1, f"{int((d > 1).sum())} elements beyond 1 bf16 ulp (max {d.max()})"
+    return err
+
+
+SHAPES = [
+    # M, N, K, fmt
+    (16, 256, 256, "nvfp4"),      # the tiny single-linear case
+    (1, 128, 256, "nvfp4"),
+    (3, 384, 768, "nvfp4"),
+    (129, 256, 1024, "nvfp4"),
+    (300, 512, 4096, "nvfp4"),
+    (128, 128, 2048, "nvfp4"),
+    (16, 256, 256, "mxfp4"),
+    (129, 384, 1024, "mxfp4"),
+]
+
+
+@pytest.mark.parametrize("M,N,K,fmt", SHAPES)
+def test_linear_matches_oracle(M, N, K, fmt):
+    X = wl.activation("laplace_outlier", 31, M + N, M, K)
+    W = wl.weight(31, N + K, N, K)
+    R = oracle.prepare(X, wl.gamma_ones(K), 1e-6, 2, 4, fmt)
+    Rw = oracle.quantize_weight(W, fmt)
+    P = upload_prepared(R, M, K, fmt)
+    w = upload_weight(Rw, N, K, fmt)
+    Y32 = sq.linear(P, w, out_fp32=True)
+    Ybf = sq.linear(P, w)
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    check(Y32, Ybf, oracle.linear(R, Rw))
+
+
+def test_linear_pipeline_through_gpu_prepare():
+    """prepare -> linear entirely on the GPU, the tiny single-linear workload."""
+    wlt = wl.WORKLOADS["tiny"]
+    lin = wlt.linears[0]
+    d = wl.linear_inputs(wlt, lin, 16)
+    P = sq.prepare(to_dev(d["X"]), to_dev(d["gamma"]), wl.EPS)
+    w = sq.quantize_weight(to_dev(d["W"]))
+    Y32 = sq.linear(P, w, out_fp32=True)
+    Ybf = sq.linear(P, w)
+    torch.cuda.synchronize()
+    R = oracle.prepare(d["X"], d["gamma"], wl.EPS)
+    Rw = oracle.quantize_weight(d["W"])
+    check(Y32, Ybf, oracle.linear(R, Rw))
+
+
+def test_linear_residual_only_and_backbone_only():
+    """Zeroing one path's codes leaves exactly the other path's product."""
+    M, N, K = 64, 256, 512
+    X = wl.activation("laplace_outlier", 32, 0, M, K)
+    W = wl.weight(32, 0, N, K)
+    R = oracle.prepare(X, wl.gamma_ones(K), 1e-6)
+    Rw = oracle.quantize_weight(W)
+    for zero in ("bb", "rs"):
+        Z = oracle.Prepared(R.mask, R.bb, R.rs, R.n, R.m, R.fmt)
+        q = getattr(R, zero)
+        setattr(Z, zero, oracle.Quantized(np.zeros_like(q.codes), q.scales, q.tscale, q.fmt))
+        P = upload_prepared(Z, M, K, "nvfp4")
+        w = upload_weight(Rw, N, K, "nvfp4")
+        Y32 = sq.linear(P, w, out_fp32=True)
+        Ybf = sq.linear(P, w)
+        torch.cuda.synchronize()
+        check(Y32, Ybf, oracle.linear(Z, Rw))
+
+
+@pytest.mark.parametrize("lin", range(4))
+def test_linear_full_size_llama_prefill_sampled(lin):
+    """Benchmark-size linears (M = 2048, Llama-3.1-8B shapes) through the GPU
+    prepare; 48 sampled rows x all N checked against the fp64 oracle."""
+    Wl = wl.WORKLOADS["llama8b"]
+    L = Wl.linears[lin]
+    d = wl.linear_inputs(Wl, L, 2048)
+    g = d["gamma"]
+    P = sq.prepare(to_dev(d["X"]), None if g is None else to_dev(g), wl.EPS)
+    w = sq.quantize_weight(to_dev(d["W"]))
+    Y32 = sq.linear(P, w, out_fp32=True)
+    Ybf = sq.linear(P, w)
+    torch.cuda.synchronize()
+    R = oracle.prepare(d["X"], g, wl.EPS)
+    Rw = oracle.quantize_weight(d["W"])
+    rows = np.sort(np.random.default_rng(lin).choice(2048, 48, replace=False))
+    check(Y32, Ybf, oracle.linear(R, Rw, rows=rows), rows=rows)
