@@ -93,8 +93,8 @@ sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps
     if (!valid_fmt(o.fmt) || !valid_shape(o.M, o.K)) return SHARQ_ERR_INVALID_ARG;
     if (!(o.m == 2 || o.m == 4 || o.m == 8) || o.n < 1 || o.n > o.m) return SHARQ_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !(eps < 1e30f)) return SHARQ_ERR_INVALID_ARG;
-    if ((o.M > 0 && !X_bf16) || !o.bb_codes || !o.bb_scales || !o.bb_tscale || !o.rs_codes ||
-        !o.rs_scales || !o.rs_tscale)
+    if (!o.bb_tscale || !o.rs_tscale) return SHARQ_ERR_INVALID_ARG;
+    if (o.M > 0 && (!X_bf16 || !o.bb_codes || !o.bb_scales || !o.rs_codes || !o.rs_scales))
         return SHARQ_ERR_INVALID_ARG;
     if (!aligned16(X_bf16) || !aligned16(gamma_bf16) || !aligned16(o.bb_codes) ||
         !aligned16(o.bb_scales) || !aligned16(o.rs_codes) || !aligned16(o.rs_scales) ||
@@ -113,12 +113,13 @@ sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps
 }
 
 static sharq_status check_linear_args(const sharq_prepared* x, const sharq_weight* w, void* Y) {
-    if (!x || !w || !Y) return SHARQ_ERR_INVALID_ARG;
+    if (!x || !w || (!Y && x->M > 0)) return SHARQ_ERR_INVALID_ARG;
     if (!valid_fmt(x->fmt) || x->fmt != w->fmt) return SHARQ_ERR_INVALID_ARG;
     if (!valid_shape(x->M, x->K) || x->K != w->K) return SHARQ_ERR_INVALID_ARG;
     if (w->N <= 0 || w->N % 128 != 0) return SHARQ_ERR_INVALID_ARG;
-    if (!x->bb_codes || !x->bb_scales || !x->bb_tscale || !x->rs_codes || !x->rs_scales ||
-        !x->rs_tscale || !w->codes || !w->scales || !w->tensor_scale)
+    if (!x->bb_tscale || !x->rs_tscale || !w->codes || !w->scales || !w->tensor_scale)
+        return SHARQ_ERR_INVALID_ARG;
+    if (x->M > 0 && (!x->bb_codes || !x->bb_scales || !x->rs_codes || !x->rs_scales))
         return SHARQ_ERR_INVALID_ARG;
     if (!aligned16(x->bb_codes) || !aligned16(x->bb_scales) || !aligned16(x->rs_codes) ||
         !aligned16(x->rs_scales) || !aligned16(w->codes) || !aligned16(w->scales) || !aligned16(Y))
@@ -130,6 +131,7 @@ sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w, void* 
                           void* stream) {
     sharq_status st = check_linear_args(x, w, Y);
     if (st != SHARQ_OK) return st;
+    if (x->M == 0) return SHARQ_OK;
     sharq::LinearLaunch p{};
     p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
     p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;

@@ -52,11 +52,17 @@ struct alignas(8) Barriers {
     uint32_t tmem_base;
 };
 
+// sf_id selects the byte inside each 32-bit scale column (two E8M0 scales
+// per MMA k-step for MXFP4): it goes into the instruction descriptor's
+// A/B scale-factor ID fields (bits 29-30 and 4-5) and into the top two bits
+// of the tensor-memory scale addresses.
 template <int FMT>
 __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
-                                    uint32_t sfb, uint32_t acc) {
-    if (FMT == 0) tc_mma_nvf4(d, a, b, Cfg<FMT>::kIdesc, sfa, sfb, acc);
-    else          tc_mma_mxf4(d, a, b, Cfg<FMT>::kIdesc, sfa, sfb, acc);
+                                    uint32_t sfb, uint32_t acc, uint32_t sf_id) {
+    const uint32_t idesc = Cfg<FMT>::kIdesc | (sf_id << 29) | (sf_id << 4);
+    const uint32_t hi = sf_id << 30;
+    if (FMT == 0) tc_mma_nvf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
+    else          tc_mma_mxf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
 }
 
 struct EpiArgs {
@@ -142,13 +148,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 for (int j = 0; j < BK / 64; ++j) {
                     const int at = j / C::kStepsPerAtom;
                     const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
-                    const uint32_t col = 4 * at, idb = sf_id << 30;
+                    const uint32_t col = 4 * at;
                     const uint64_t db = sdesc_sw128(a_w + 32 * j);
                     const uint32_t acc = (kb | j) ? 1u : 0u;
-                    mma<FMT>(t_acc_b, sdesc_sw128(a_b + 32 * j), db, (t_sfa_b + col) | idb,
-                             (t_sfb + col) | idb, acc);
-                    mma<FMT>(t_acc_r, sdesc_sw128(a_r + 32 * j), db, (t_sfa_r + col) | idb,
-                             (t_sfb + col) | idb, acc);
+                    mma<FMT>(t_acc_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + col,
+                             acc, sf_id);
+                    mma<FMT>(t_acc_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + col,
+                             acc, sf_id);
                 }
                 tc_commit(&bars->empty[s]);
             }

@@ -254,6 +254,16 @@ def linear(prep: Prepared, w: Quantized, rows: Optional[np.ndarray] = None,
     return float(w.tscale) * (float(prep.bb.tscale) * Sb + float(prep.rs.tscale) * Sr)
 
 
+def linear_abs(prep: Prepared, w: Quantized, rows: Optional[np.ndarray] = None) -> np.ndarray:
+    """G_w * (G_b |Db| |Dw|^T + G_r |Dr| |Dw|^T) in fp64: the magnitude sum
+    that bounds the rounding error of any fp32 accumulation of the linear
+    (recursive summation: |error| <= gamma_n * sum |a_k b_k|)."""
+    Db = np.abs(dequant_blocks(prep.bb, rows))
+    Dr = np.abs(dequant_blocks(prep.rs, rows))
+    Dw = np.abs(dequant_blocks(w))
+    return float(w.tscale) * (float(prep.bb.tscale) * (Db @ Dw.T) + float(prep.rs.tscale) * (Dr @ Dw.T))
+
+
 def gather_rows(prep: Prepared, row_index: np.ndarray) -> Prepared:
     """The prepared rows a grouped linear reads, in dispatch order (tensor
     scales stay those of the whole prepare call)."""
