@@ -256,8 +256,14 @@ cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s) {
         return cudaErrorInvalidValue;
     const size_t smem = kStages * C::kStageStride + sizeof(Barriers) + 1024;
     auto kfn = linear_kernel<FMT>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
     dim3 grid((unsigned)((p.M + BM - 1) / BM), (unsigned)(p.N / BN));
     kfn<<<grid, kThreads, smem, s>>>(tb, tr, tw, static_cast<const uint8_t*>(p.bb_scales),

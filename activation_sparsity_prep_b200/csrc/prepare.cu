@@ -378,18 +378,28 @@ prepare_kernel(PrepArgs a) {
 template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT>;
+    static int blocks_per_sm = 0;          // same for every device of one architecture
+    if (blocks_per_sm == 0) {
+        int b = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kfn, kThreads, 0);
+        if (e != cudaSuccess) return e;
+        blocks_per_sm = b;
+    }
     int64_t Mpad = (a.M + 127) / 128 * 128;
     int64_t want = (Mpad + kWarps - 1) / kWarps;
-    int blocks_per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kfn, kThreads, 0);
-    if (e != cudaSuccess) return e;
     int64_t cap = (int64_t)blocks_per_sm * max_blocks;
     int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
-    PrepArgs args = a;
-    void* params[] = {&args};
-    if (FMT == 0)   // two grid-wide barriers: all blocks must be co-resident
-        return cudaLaunchCooperativeKernel((const void*)kfn, dim3(grid), dim3(kThreads), params, 0, s);
-    return cudaLaunchKernel((const void*)kfn, dim3(grid), dim3(kThreads), params, 0, s);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // grid barriers: all blocks co-resident
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (FMT == 0) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kfn, a);
 }
 
 template <int FMT, bool HAS_GAMMA, bool WEIGHT>

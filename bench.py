@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the SharQ hot path on B200.
+
+One step = the four linears of a Llama-3.1-8B-shaped decoder layer (qkv,
+o, gate+up, down) at prefill M = 2048 tokens, each run as the fused
+prepare (RMSNorm + 2:4 mask + NVFP4 backbone + NVFP4 residual) followed by
+the two-path tcgen05 FP4 linear.  Weights are quantised once, outside the
+timed region.  Inputs are seeded synthetic tensors (Laplace activations with
+0.5 % outlier channels, N(0, 0.02) weights).
+
+Metric: effective TFLOP/s = sum over linears of 2*M*N*K / step time; the
+JSON line also carries tokens/s, the roofline of the dominant kernel (the
+FP4 linear) and of the prepare kernel, the CPU oracle baseline, the SM
+clocks seen during the timed region and an end-to-end figure with host
+buffers.  ``--impl reference`` times the CPU oracle instead.
+
+Multi-GPU: the path has no exchange step at this scale; each rank runs an
+independent replica (weak scaling) and the slowest rank's time counts.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from activation_sparsity_prep_b200 import workloads as wl  # noqa: E402
+
+METRIC = "SharQ linear eff. TFLOPS & tokens/s, % of FP4 roofline; prep kernel HBM GB/s"
+L2_FLUSH_BYTES = 512 << 20          # > 126 MB L2
+PREP_BYTES_PER_ELEM = {(0, 1): 3.125, (1, 1): 3.0625}   # (fmt, zero-filled backbone)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--fmt", default="nvfp4")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def rank_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- inputs ----
+
+def make_inputs(W: wl.Workload, M: int):
+    out = []
+    for L in W.linears:
+        d = wl.linear_inputs(W, L, M)
+        out.append((L, d))
+    return out
+
+
+def flops_of(linears, M):
+    return sum(2.0 * M * L.N * L.K for L, _ in linears)
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "activation_sparsity_prep_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(launch_key: str, sha: str):
+    """DRAM bytes (read + write) of this exact launch from the committed ncu
+    summary, or None when the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)[launch_key]
+    except Exception:
+        return None
+    if t.get("source_sha") != sha:
+        return None
+    return t["dram_bytes"]
+
+
+# ------------------------------------------------------------ CPU arm ----
+
+def oracle_sample_step(linears, rows: int, quantized):
+    """One bounded oracle step: prepare and linear of the first `rows` rows
+    of every linear.  Returns (seconds, effective flops of the sample)."""
+    import oracle
+    t0 = time.perf_counter()
+    fl = 0.0
+    for (L, d), Wq in zip(linears, quantized):
+        P = oracle.prepare(d["X"][:rows], d["gamma"], wl.EPS)
+        oracle.linear(P, Wq)
+        fl += 2.0 * rows * L.N * L.K
+    return time.perf_counter() - t0, fl
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(linears, budget_s: float = 15.0, rows: int = 16):
+    import oracle
+    quantized = [oracle.quantize_weight(d["W"]) for _, d in linears]
+    total_t, total_f, n = 0.0, 0.0, 0
+    while total_t < budget_s and n < 50:
+        t, f = oracle_sample_step(linears, rows, quantized)
+        total_t += t
+        total_f += f
+        n += 1
+    return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} passes of: oracle prepare + fp64 two-path linear on the first {rows} "
+                      f"rows of each of the 4 linears (all N); prepare single-threaded C, "
+                      f"GEMM numpy/OpenBLAS fp64"}
+
+
+def run_reference(args):
+    rank, world, _ = rank_info()
+    if rank != 0:
+        return 0
+    W = wl.WORKLOADS[args.workload]
+    linears = make_inputs(W, args.M)
+    import oracle
+    quantized = [oracle.quantize_weight(d["W"]) for _, d in linears]
+    rows = 16
+    for _ in range(args.warmup):
+        oracle_sample_step(linears, rows, quantized)
+    times, fl = [], 0.0
+    for _ in range(args.steps):
+        t, f = oracle_sample_step(linears, rows, quantized)
+        times.append(t)
+        fl = f
+    tot = sum(times)
+    value = fl * args.steps / tot / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 GEMM over FP4-decoded operands; f32 prepare",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload} decoder linears, sample of {rows} rows per linear "
+                               f"(of M={args.M})", "M_sampled": rows, "fmt": "nvfp4", "nm": "2:4"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {rows} rows of each linear per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU arm ----
+
+def run_sharq(args):
+    import torch
+    import torch.distributed as dist
+
+    import activation_sparsity_prep_b200 as sq
+
+    rank, world, local = rank_info()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    W = wl.WORKLOADS[args.workload]
+    M = args.M
+    fmt = sq._FMT[args.fmt]
+    linears = make_inputs(W, M)
+
+    # device buffers
+    bufs = []
+    for L, d in linears:
+        X = torch.from_numpy(d["X"]).view(torch.bfloat16).to(dev)
+        g = None if d["gamma"] is None else torch.from_numpy(d["gamma"]).view(torch.bfloat16).to(dev)
+        Wt = torch.from_numpy(d["W"]).view(torch.bfloat16).to(dev)
+        w = sq.quantize_weight(Wt, fmt)
+        del Wt
+        P = sq.Prepared.empty(M, L.K, 2, 4, fmt, device=dev)
+        ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
+        Y = torch.empty((M, L.N), dtype=torch.bfloat16, device=dev)
+        bufs.append(dict(L=L, X=X, g=g, w=w, P=P, ws=ws, Y=Y))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        for b in bufs:
+            sq.prepare(b["X"], b["g"], wl.EPS, 2, 4, fmt, out=b["P"], ws=b["ws"])
+            sq.linear(b["P"], b["w"], out=b["Y"])
+
+    # eager warm-up (lazy init), then capture one step with per-kernel events
+    step()
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    nev = 2 * len(bufs) + 1
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)]
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            evs[0].record()
+            for i, b in enumerate(bufs):
+                sq.prepare(b["X"], b["g"], wl.EPS, 2, 4, fmt, out=b["P"], ws=b["ws"])
+                evs[2 * i + 1].record()
+                sq.linear(b["P"], b["w"], out=b["Y"])
+                evs[2 * i + 2].record()
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, prep_ms, lin_ms = [], [[] for _ in bufs], [[] for _ in bufs]
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            flush.zero_()                    # L2 flushed between timed steps
+            g.replay()
+            torch.cuda.synchronize()
+            step_ms.append(evs[0].elapsed_time(evs[-1]))
+            for i in range(len(bufs)):
+                prep_ms[i].append(evs[2 * i].elapsed_time(evs[2 * i + 1]))
+                lin_ms[i].append(evs[2 * i + 1].elapsed_time(evs[2 * i + 2]))
+    torch.cuda.synchronize()
+    status = sq.last_device_status()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    clocks = clk.summary()
+
+    fl_step = flops_of(linears, M)
+    ms_step = total_ms / args.steps
+    value = fl_step * world * args.steps / (total_ms * 1e-3) / 1e12
+    tokens = M * world * args.steps / (total_ms * 1e-3)
+
+    hbm, bf16, src = peaks()
+    fp4_peak = 4.0 * bf16           # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PFLOP/s)
+    lin_t = [statistics.mean(x) * 1e-3 for x in lin_ms]
+    prep_t = [statistics.mean(x) * 1e-3 for x in prep_ms]
+    # Dominant kernel: the largest linear launch (gate+up).  Algorithmic
+    # dense-equivalent flops of the two-path linear at 2:4: 2MNK on the dense
+    # residual plus 2MNK*(n/m) on the sparse backbone at twice the rate.
+    dom = max(range(len(bufs)), key=lambda i: lin_t[i])
+    Ld = bufs[dom]["L"]
+    achieved = 2.5 * M * Ld.N * Ld.K / lin_t[dom] / 1e12
+    traffic = profiled_traffic(f"linear_{args.fmt}_{W.name}_{Ld.name}_M{M}",
+                               source_sha("linear.cu", "common.cuh"))
+    # Prepare roofline on its largest launch (algorithmic bytes per element:
+    # read X 2, backbone codes 0.5 (zero-filled) + scales, residual codes 0.5 + scales)
+    pdom = max(range(len(bufs)), key=lambda i: prep_t[i])
+    Lp = bufs[pdom]["L"]
+    prep_ach = PREP_BYTES_PER_ELEM[(fmt, 1)] * M * Lp.K / prep_t[pdom] / 1e9
+    prep_traffic = profiled_traffic(f"prepare_{args.fmt}_{W.name}_{Lp.name}_M{M}",
+                                    source_sha("prepare.cu", "common.cuh"))
+
+    # end-to-end: host inputs (pinned) in, host outputs out, every step
+    e2e = None
+    if not args.no_e2e:
+        hx = [b["X"].cpu().pin_memory() for b in bufs]
+        hy = [torch.empty(b["Y"].shape, dtype=b["Y"].dtype, pin_memory=True) for b in bufs]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        cur = torch.cuda.current_stream()
+        for it in range(args.warmup + args.steps):
+            flush.zero_()
+            e0.record(cur)
+            for b, h in zip(bufs, hx):
+                b["X"].copy_(h, non_blocking=True)
+            g.replay()
+            for b, h in zip(bufs, hy):
+                h.copy_(b["Y"], non_blocking=True)
+            e1.record(cur)
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                ts.append(e0.elapsed_time(e1))
+        tot = sum(ts)
+        if world > 1:
+            t = torch.tensor([tot], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            tot = float(t.item())
+        e2e = {"value": fl_step * world * args.steps / (tot * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hx)),
+               "d2h_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hy)),
+               "ms_per_step": tot / args.steps}
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(linears)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4" if fmt == 0 else "mxfp4", "data": "synthetic",
+            "config": {"workload": f"{W.name}: Llama-3.1-8B-shaped decoder linears "
+                                   f"(qkv 4096x6144, o 4096x4096, gate_up 4096x28672, "
+                                   f"down 14336x4096), prefill M={M}, prepare+linear each",
+                       "M": M, "fmt": args.fmt, "nm": "2:4", "rmsnorm": "qkv, gate_up",
+                       "l2": "flushed between timed steps (512 MiB write)",
+                       "timing": "CUDA graph per step, per-kernel external events"},
+            "tokens_per_s": tokens,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic,
+                         "kernel": f"linear_kernel (two-path FP4 GEMM), {Ld.name} launch "
+                                   f"M={M} N={Ld.N} K={Ld.K}",
+                         "peak_note": f"dense FP4 = 4 x {src} bf16 burst ({bf16:.0f} TFLOP/s)",
+                         "achieved_note": "2.5*M*N*K per launch (2:4 backbone at 2x rate + dense residual)"},
+            "prepare_roofline": {"bound": "hbm", "achieved": prep_ach, "peak": hbm, "unit": "GB/s",
+                                 "frac": prep_ach / hbm, "traffic": prep_traffic,
+                                 "kernel": f"prepare_kernel, {Lp.name} launch M={M} K={Lp.K}",
+                                 "bytes_per_elem": PREP_BYTES_PER_ELEM[(fmt, 1)],
+                                 "peak_note": f"{src} copy bandwidth"},
+            "kernel_ms": {b["L"].name: {"prepare": statistics.mean(p), "linear": statistics.mean(l)}
+                          for b, p, l in zip(bufs, prep_ms, lin_ms)},
+            "executed_fp4_tflops": sum(4.0 * M * b["L"].N * b["L"].K for b in bufs) / sum(lin_t) / 1e12,
+            "prepare_gbs_all": sum(PREP_BYTES_PER_ELEM[(fmt, 1)] * M * b["L"].K for b in bufs) / sum(prep_t) / 1e9,
+            "gpu_launches": 2 * len(bufs) * args.steps,
+            "device_status": status,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_sharq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
