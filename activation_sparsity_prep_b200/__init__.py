@@ -21,7 +21,7 @@ from typing import Optional
 __all__ = [
     "NVFP4", "MXFP4", "SharqError", "load_sharq_ops", "scale_bytes",
     "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
-    "prepare", "linear", "moe_linear", "last_device_status",
+    "prepare", "prepare_noalloc", "linear", "moe_linear", "last_device_status",
 ]
 
 NVFP4, MXFP4 = 0, 1
@@ -88,6 +88,8 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_moe_linear.argtypes = [ctypes.POINTER(_Prepared), P, P, I, I64,
                                        ctypes.POINTER(_Weight), P, I, P]
         L.sharq_moe_linear.restype = I
+        L.sharq_prepare_noalloc.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P]
+        L.sharq_prepare_noalloc.restype = I
         L.sharq_last_device_status.argtypes = [P]
         L.sharq_last_device_status.restype = I
         _lib = L
@@ -218,6 +220,25 @@ def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4
     _check("sharq_prepare",
            L.sharq_prepare(X.data_ptr(), _ptr(gamma), float(eps), ctypes.byref(cp),
                            ws.data_ptr(), ws.numel(), _stream(stream)))
+    return p
+
+
+NOALLOC_MAX_ROWS = 262144
+
+
+def prepare_noalloc(X, gamma=None, eps: float = 1e-6, out: Optional[Prepared] = None,
+                    n: int = 2, m: int = 4, fmt="nvfp4", stream=None) -> Prepared:
+    """prepare() through the entry point that allocates no device memory
+    (fixed in-library scratch, M <= NOALLOC_MAX_ROWS).  The output buffers
+    are the caller's: pass ``out`` when the caller cannot allocate either."""
+    L = load_sharq_ops()
+    M, K = X.shape
+    f = _fmt(fmt)
+    p = out if out is not None else Prepared.empty(M, K, n, m, f, device=X.device)
+    cp = p._c()
+    _check("sharq_prepare_noalloc",
+           L.sharq_prepare_noalloc(X.data_ptr(), _ptr(gamma), float(eps), ctypes.byref(cp),
+                                   _stream(stream)))
     return p
 
 

@@ -156,6 +156,31 @@ SHARQ_API sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* 
                               const sharq_weight* w, void* Y, int y_is_fp32,
                               void* stream);
 
+/* Largest M that sharq_prepare_noalloc() accepts (its fixed scratch array
+ * holds 64 bytes plus 4 bytes per row: 1 MiB + 64 bytes in all). */
+#define SHARQ_NOALLOC_MAX_ROWS 262144
+
+/* sharq_prepare without a workspace argument, for callers that cannot
+ * allocate device memory where they run it: work enqueued during CUDA graph
+ * stream capture, plugin or runtime callbacks whose host framework owns all
+ * device memory, and serving loops that cannot pay for the device-wide
+ * synchronisation of cudaMalloc/cudaFree.  The paper has no counterpart;
+ * this is a deployment variant of the preparation operator above, with the
+ * same arguments (minus ws) and bit-identical outputs.
+ *   - Scratch lives in a fixed array inside the library (64 + 4 * M bytes,
+ *     at most SHARQ_NOALLOC_MAX_ROWS rows).  Every GPU that loads the library
+ *     holds that array until the process exits.
+ *   - M > SHARQ_NOALLOC_MAX_ROWS returns SHARQ_ERR_INVALID_ARG.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race on it.  Each call clears the part
+ *     that must start at zero.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+SHARQ_API sharq_status sharq_prepare_noalloc(const void* X_bf16, const void* gamma_bf16, float eps,
+                                             const sharq_prepared* out, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word:
  * SHARQ_OK, SHARQ_ERR_TIMEOUT if a bounded device wait gave up since the
  * last call, or SHARQ_ERR_CUDA if the stream itself reports an error. */
