@@ -8,11 +8,12 @@
 //   phase 2  mask, backbone codes/scales with G_b, residual r,
 //            A_r = max|r|                                 -> grid barrier
 //   phase 3  residual codes/scales with G_r
-// One persistent cooperative launch runs the three phases; each warp owns
-// whole rows, lane l reading the 16-byte chunks l, l+32, ... of a row, which
-// is also the fixed fp32 reduction order of the RMS sum.  MXFP4 has no
-// tensor scale, so its backbone and residual are produced in one pass with
-// no barrier.
+// One persistent cooperative launch runs the three phases.  In phase 1 each
+// warp owns whole rows, lane l reading the 16-byte chunks l, l+32, ... of a
+// row, which is also the fixed fp32 reduction order of the RMS sum; phases 2
+// and 3 spread (row, 256-element segment) items over every warp.  MXFP4 has
+// no tensor scale, so its backbone and residual are produced in one pass
+// (after the RMS barrier when there is a norm).
 //
 // Every floating-point step is one correctly rounded fp32 operation
 // (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn, no contraction), so the
@@ -102,11 +103,16 @@ __device__ __forceinline__ uint32_t topn_bits(const float y[8], int n) {
     return bits;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ float amax8(const float v[8]) {
-    float m = 0.0f;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) m = fmaxf(m, fabsf(v[t]));
-    return m;
+    float m0 = max3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+    float m1 = max3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+    return max3(m0, m1, fmaxf(fabsf(v[6]), fabsf(v[7])));
 }
 
 // 2^p as fp32 for -127 <= p <= 127 (2^-127 is subnormal).
@@ -187,25 +193,112 @@ __device__ __forceinline__ void fill_inv_table(float* tab, float genc) {
     __syncthreads();
 }
 
-// Gather 4 consecutive block-scale bytes into one word at lane `lead` of each
-// group of `stride*4` lanes: word = v(lead) | v(lead+stride)<<8 | ...
-__device__ __forceinline__ uint32_t gather4(uint32_t v, int lane, int stride) {
-    int lead = lane & ~(4 * stride - 1);
-    uint32_t w = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) w |= __shfl_sync(0xffffffffu, v, lead + q * stride) << (8 * q);
-    return w;
+// ------------------------------------------------------------------------
+// Phases 2 and 3 give each lane one whole scale block (16 elements for
+// NVFP4, 32 for MXFP4) of the flattened [M, K/BS] block array.  A warp's 32
+// blocks are 32*BS consecutive elements of X, so its loads stay coalesced;
+// the block maximum needs no shuffle, and a lane stores its codes with one
+// 8- or 16-byte store and its scale with one byte store.  Neither phase has
+// an ordering constraint (block-local arithmetic plus an exact maximum).
+// ------------------------------------------------------------------------
+
+// Walk the blocks b = start, start + stride, ... as (row, column) pairs
+// without a division per step.
+struct BlockCursor {
+    int64_t row;
+    int cb;
+    int dr, dc, nbr;
+    __device__ __forceinline__ void init(int64_t start, int64_t stride, int nb_row) {
+        nbr = nb_row;
+        row = start / nb_row;
+        cb = (int)(start - row * nb_row);
+        dr = (int)(stride / nb_row);
+        dc = (int)(stride - (int64_t)dr * nb_row);
+    }
+    __device__ __forceinline__ void next() {
+        cb += dc;
+        row += dr;
+        if (cb >= nbr) { cb -= nbr; ++row; }
+    }
+};
+
+// Element i of a group of four is kept when it beats at least two of the
+// other three (a beats b: |a| > |b|, or equal and a has the lower index).
+__device__ __forceinline__ uint32_t keep_2of4(const float* y) {
+    const float a0 = fabsf(y[0]), a1 = fabsf(y[1]), a2 = fabsf(y[2]), a3 = fabsf(y[3]);
+    const bool b01 = a0 >= a1, b02 = a0 >= a2, b03 = a0 >= a3;
+    const bool b12 = a1 >= a2, b13 = a1 >= a3, b23 = a2 >= a3;
+    const bool k0 = (b01 & b02) | (b01 & b03) | (b02 & b03);
+    const bool k1 = (!b01 & b12) | (!b01 & b13) | (b12 & b13);
+    const bool k2 = (!b02 & !b12) | (!b02 & b23) | (!b12 & b23);
+    const bool k3 = (!b03 & !b13) | (!b03 & !b23) | (!b13 & !b23);
+    return (uint32_t)k0 | ((uint32_t)k1 << 1) | ((uint32_t)k2 << 2) | ((uint32_t)k3 << 3);
 }
+
+// Keep bits of E consecutive elements (E a multiple of 8).
+template <int E, int MG, bool NM24>
+__device__ __forceinline__ uint32_t keep_bits(const float* y, int n) {
+    uint32_t k = 0;
+#pragma unroll
+    for (int g = 0; g < E; g += (NM24 ? 4 : 8)) {
+        if (NM24) k |= keep_2of4(y + g) << g;
+        else      k |= topn_bits<MG>(y + g, n) << g;
+    }
+    return k;
+}
+
+template <int E>
+__device__ __forceinline__ float amaxE(const float* v) {
+    float m = amax8(v);
+#pragma unroll
+    for (int g = 8; g < E; g += 8) m = fmaxf(m, amax8(v + g));
+    return m;
+}
+
+template <int FMT, bool HAS_GAMMA>
+struct LaneBlock {
+    static constexpr int E = FMT == 0 ? 16 : 32;   // elements per lane = one scale block
+    static constexpr int NV = E / 8;                // 16-byte chunks
+    uint4 x[NV];
+    uint4 g[NV];
+    float rinv;
+
+    __device__ __forceinline__ void load(const PrepArgs& a, int64_t row, int cb, const float* rinv_ws) {
+        const uint16_t* xp = a.X + row * a.K + (int64_t)cb * E;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) x[v] = ld_nc_v4(xp + 8 * v);
+        if (HAS_GAMMA) {
+#pragma unroll
+            for (int v = 0; v < NV; ++v) g[v] = ld_nc_v4(a.gamma + (int64_t)cb * E + 8 * v);
+            rinv = rinv_ws[row];
+        }
+    }
+
+    __device__ __forceinline__ void y(float* out) const {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            unpack_bf16x8(x[v], out + 8 * v);
+            if (HAS_GAMMA) {
+                float gg[8];
+                unpack_bf16x8(g[v], gg);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) out[8 * v + t] = __fmul_rn(__fmul_rn(out[8 * v + t], rinv), gg[t]);
+            }
+        }
+    }
+};
 
 // ------------------------------------------------------------------------
 // The kernel.  FMT: 0 NVFP4, 1 MXFP4.  WEIGHT: quantise the whole tensor
-// once (keep-all, no norm, no residual).
+// once (keep-all, no norm, no residual).  NM24: the 2-of-4 mask.
 // ------------------------------------------------------------------------
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT>
-__global__ void __launch_bounds__(kThreads)
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24>
+__global__ void __launch_bounds__(kThreads, 2)
 prepare_kernel(PrepArgs a) {
     __shared__ float s_inv[128];
     __shared__ float s_red[kWarps];
+    using LB = LaneBlock<FMT, HAS_GAMMA>;
+    constexpr int E = LB::E;
 
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -219,17 +312,29 @@ prepare_kernel(PrepArgs a) {
     float* rinv_ws = ws_rinv(a.ws);
 
     // ---------------- phase 1: rinv per row, A_b = max |y| ----------------
+    // One warp per row: lane l adds the squares of chunks l, l+32, ... in k
+    // order (the fixed reduction order), eight chunk loads in flight per lane.
     float amax = 0.0f;
     if (HAS_GAMMA || FMT == 0) {
         for (int64_t row = gwarp; row < M; row += nwarps) {
+            const uint16_t* xr = a.X + row * K;
             float rinv = 1.0f;
             if (HAS_GAMMA) {
                 float acc = 0.0f;
-                for (int c = lane; c < nchunk; c += 32) {
-                    float x[8];
-                    unpack_bf16x8(ld_nc_v4(a.X + row * K + (int64_t)c * 8), x);
+                for (int c0 = lane; c0 < nchunk; c0 += 256) {
+                    uint4 v[8];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, __fmul_rn(x[t], x[t]));
+                    for (int u = 0; u < 8; ++u)
+                        if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (c0 + 32 * u < nchunk) {
+                            float x[8];
+                            unpack_bf16x8(v[u], x);
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, __fmul_rn(x[t], x[t]));
+                        }
+                    }
                 }
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1)
@@ -239,10 +344,48 @@ prepare_kernel(PrepArgs a) {
                 if (lane == 0) rinv_ws[row] = rinv;
             }
             if (FMT == 0) {
-                for (int c = lane; c < nchunk; c += 32) {
-                    float y[8];
-                    load_y<HAS_GAMMA>(a, row, c, rinv, y);
-                    amax = fmaxf(amax, amax8(y));
+                if (HAS_GAMMA) {
+                    for (int c0 = lane; c0 < nchunk; c0 += 128) {
+                        uint4 v[4], g[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (c0 + 32 * u < nchunk) {
+                                v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+                                g[u] = ld_nc_v4(a.gamma + (int64_t)(c0 + 32 * u) * 8);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (c0 + 32 * u < nchunk) {
+                                float y[8], gg[8];
+                                unpack_bf16x8(v[u], y);
+                                unpack_bf16x8(g[u], gg);
+#pragma unroll
+                                for (int t = 0; t < 8; ++t) y[t] = __fmul_rn(__fmul_rn(y[t], rinv), gg[t]);
+                                amax = fmaxf(amax, amax8(y));
+                            }
+                        }
+                    }
+                } else {
+                    // y = x: the magnitude order of bf16 values is the integer
+                    // order of their bits with the sign cleared.
+                    uint32_t m2 = 0;
+                    for (int c0 = lane; c0 < nchunk; c0 += 256) {
+                        uint4 v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (c0 + 32 * u < nchunk) {
+                                m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
+                                m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
+                                m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
+                                m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+                            }
+                        }
+                    }
+                    amax = fmaxf(amax, fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u)));
                 }
             }
         }
@@ -252,8 +395,7 @@ prepare_kernel(PrepArgs a) {
         block_amax_to_global(amax, &a.ws[0], s_red);
         grid_barrier(&a.ws[2], gridDim.x);
     } else if (HAS_GAMMA) {
-        __syncthreads();
-        if (threadIdx.x == 0) __threadfence();
+        grid_barrier(&a.ws[2], gridDim.x);   // rinv of every row visible to every warp
     }
 
     // ------- phase 2: mask, backbone, residual amax (and MXFP4 residual) -------
@@ -269,28 +411,38 @@ prepare_kernel(PrepArgs a) {
         }
     }
 
-    float ramax = 0.0f;
-    for (int64_t row = gwarp; row < Mpad; row += nwarps) {
-        if (row >= M) {   // padding rows of the scale atoms carry zero scales
-            for (int s4 = lane; s4 < nsf / 4; s4 += 32) {
-                *reinterpret_cast<uint32_t*>(a.bb_scales + sf_off(row, s4 * 4, nsf)) = 0u;
-                if (!WEIGHT)
-                    *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, s4 * 4, nsf)) = 0u;
-            }
-            continue;
+    // padding rows of the scale atoms carry zero scales
+    {
+        const int words = nsf / 4;
+        const int64_t npad = (Mpad - M) * words;
+        for (int64_t i = gwarp * 32 + lane; i < npad; i += nwarps * 32) {
+            const int64_t row = M + i / words;
+            const int s4 = (int)(i % words);
+            *reinterpret_cast<uint32_t*>(a.bb_scales + sf_off(row, s4 * 4, nsf)) = 0u;
+            if (!WEIGHT) *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, s4 * 4, nsf)) = 0u;
         }
-        const float rinv = HAS_GAMMA ? rinv_ws[row] : 1.0f;
-        for (int c = lane; c < nchunk; c += 32) {
-            float y[8];
-            load_y<HAS_GAMMA>(a, row, c, rinv, y);
-            uint32_t keep = WEIGHT ? 0xFFu : topn_bits<MG>(y, a.n);
-            float B[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) B[t] = ((keep >> t) & 1u) ? y[t] : 0.0f;
-            float bm = amax8(B);
-            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-            if (FMT == 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+    }
 
+    const int nb_row = K / E;
+    float ramax = 0.0f;
+    {
+        BlockCursor cur;
+        cur.init(gwarp * 32 + lane, nwarps * 32, nb_row);
+        LB lb;
+        if (cur.row < M) lb.load(a, cur.row, cur.cb, rinv_ws);
+        while (cur.row < M) {
+            BlockCursor nxt = cur;
+            nxt.next();
+            LB ln;
+            if (nxt.row < M) ln.load(a, nxt.row, nxt.cb, rinv_ws);   // prefetch
+
+            const int64_t row = cur.row;
+            const int cb = cur.cb;
+            float y[E];
+            lb.y(y);
+            // the backbone's block max is the block max of y: the largest
+            // entry of every group is always kept
+            const float bm = amaxE<E>(y);
             uint32_t ecode;
             float inv, sdec;
             if (FMT == 0) {
@@ -302,41 +454,56 @@ prepare_kernel(PrepArgs a) {
                 inv = pow2f(127 - (int)ecode);
                 sdec = pow2f((int)ecode - 127);
             }
-            float t8[8];
+            const uint32_t keep = WEIGHT ? 0xFFFFFFFFu : keep_bits<E, MG, NM24>(y, a.n);
+            uint32_t codes[E / 8];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(B[t], inv);
-            uint32_t codes = cvt_e2m1x8(t8);
-            *reinterpret_cast<uint32_t*>(a.bb_codes + row * (K / 2) + (int64_t)c * 4) = codes;
-            if (a.mask && !WEIGHT) a.mask[row * (K / 8) + c] = (uint8_t)keep;
-
-            const int stride = (FMT == 0) ? 2 : 4;
-            uint32_t word = gather4(ecode, lane, stride);
-            if ((lane & (4 * stride - 1)) == 0)
-                *reinterpret_cast<uint32_t*>(a.bb_scales + sf_off(row, (c * 8) / BS, nsf)) = word;
+            for (int v = 0; v < E / 8; ++v) {
+                float t8[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    t8[t] = ((keep >> (8 * v + t)) & 1u) ? __fmul_rn(y[8 * v + t], inv) : 0.0f;
+                codes[v] = cvt_e2m1x8(t8);
+            }
+            uint8_t* cp = a.bb_codes + row * (K / 2) + (int64_t)cb * (E / 2);
+            if (E == 16) *reinterpret_cast<uint2*>(cp) = make_uint2(codes[0], codes[1]);
+            else         *reinterpret_cast<uint4*>(cp) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            a.bb_scales[sf_off(row, cb, nsf)] = (uint8_t)ecode;
+            if (!WEIGHT && a.mask) {
+                uint8_t* mp = a.mask + row * (K / 8) + (int64_t)cb * (E / 8);
+                if (E == 16) *reinterpret_cast<uint16_t*>(mp) = (uint16_t)keep;
+                else         *reinterpret_cast<uint32_t*>(mp) = keep;
+            }
 
             if (!WEIGHT) {
-                float d[8], r[8];
-                dequant8(codes, sdec, sb.gdec, d);
+                // residual r = y - dequant(backbone), in place in y
 #pragma unroll
-                for (int t = 0; t < 8; ++t) r[t] = __fsub_rn(y[t], d[t]);
+                for (int v = 0; v < E / 8; ++v) {
+                    float d[8];
+                    dequant8(codes[v], sdec, sb.gdec, d);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) y[8 * v + t] = __fsub_rn(y[8 * v + t], d[t]);
+                }
                 if (FMT == 0) {
-                    ramax = fmaxf(ramax, amax8(r));
+                    ramax = fmaxf(ramax, amaxE<E>(y));
                 } else {
                     // MXFP4: the residual needs no tensor-wide scale; finish it here.
-                    float rm = amax8(r);
-                    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 1));
-                    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 2));
-                    uint32_t rc = mx_code(rm);
-                    float rinvs = pow2f(127 - (int)rc);
+                    const uint32_t rcode = mx_code(amaxE<E>(y));
+                    const float rs = pow2f(127 - (int)rcode);
+                    uint32_t rc[E / 8];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) r[t] = __fmul_rn(r[t], rinvs);
-                    *reinterpret_cast<uint32_t*>(a.rs_codes + row * (K / 2) + (int64_t)c * 4) =
-                        cvt_e2m1x8(r);
-                    uint32_t rw = gather4(rc, lane, 4);
-                    if ((lane & 15) == 0)
-                        *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, (c * 8) / 32, nsf)) = rw;
+                    for (int v = 0; v < E / 8; ++v) {
+                        float t8[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[8 * v + t], rs);
+                        rc[v] = cvt_e2m1x8(t8);
+                    }
+                    *reinterpret_cast<uint4*>(a.rs_codes + row * (K / 2) + (int64_t)cb * (E / 2)) =
+                        make_uint4(rc[0], rc[1], rc[2], rc[3]);
+                    a.rs_scales[sf_off(row, cb, nsf)] = (uint8_t)rcode;
                 }
             }
+            cur = nxt;
+            lb = ln;
         }
     }
     if (FMT == 1 || WEIGHT) return;
@@ -349,35 +516,62 @@ prepare_kernel(PrepArgs a) {
     __syncthreads();                       // everyone done reading the backbone table
     fill_inv_table(s_inv, sr.genc);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.rs_tscale = sr.gdec;
-    for (int64_t row = gwarp; row < M; row += nwarps) {
-        const float rinv = HAS_GAMMA ? rinv_ws[row] : 1.0f;
-        for (int c = lane; c < nchunk; c += 32) {
-            float y[8];
-            load_y<HAS_GAMMA>(a, row, c, rinv, y);
-            // backbone dequant from the codes and scale written in phase 2
-            uint32_t codes = *reinterpret_cast<const uint32_t*>(a.bb_codes + row * (K / 2) + (int64_t)c * 4);
-            uint32_t eb = a.bb_scales[sf_off(row, c / 2, nsf)];
-            float d[8], r[8];
-            dequant8(codes, e4m3_to_f32(eb), sb.gdec, d);
+    {
+        BlockCursor cur;
+        cur.init(gwarp * 32 + lane, nwarps * 32, nb_row);
+        LB lb;
+        uint2 bc = make_uint2(0, 0);
+        uint32_t bs = 0;
+        if (cur.row < M) {
+            lb.load(a, cur.row, cur.cb, rinv_ws);
+            bc = *reinterpret_cast<const uint2*>(a.bb_codes + cur.row * (K / 2) + (int64_t)cur.cb * 8);
+            bs = a.bb_scales[sf_off(cur.row, cur.cb, nsf)];
+        }
+        while (cur.row < M) {
+            BlockCursor nxt = cur;
+            nxt.next();
+            LB ln;
+            uint2 nbc = make_uint2(0, 0);
+            uint32_t nbs = 0;
+            if (nxt.row < M) {
+                ln.load(a, nxt.row, nxt.cb, rinv_ws);
+                nbc = *reinterpret_cast<const uint2*>(a.bb_codes + nxt.row * (K / 2) + (int64_t)nxt.cb * 8);
+                nbs = a.bb_scales[sf_off(nxt.row, nxt.cb, nsf)];
+            }
+            const int64_t row = cur.row;
+            const int cb = cur.cb;
+            float y[16];
+            lb.y(y);
+            const float sdec = e4m3_to_f32(bs);
+            float d[8];
+            dequant8(bc.x, sdec, sb.gdec, d);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) r[t] = __fsub_rn(y[t], d[t]);
-            float rm = amax8(r);
-            rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 1));
-            uint32_t er = cvt_e4m3(__fmul_rn(rm, sr.k1));
-            float inv = s_inv[er];
+            for (int t = 0; t < 8; ++t) y[t] = __fsub_rn(y[t], d[t]);
+            dequant8(bc.y, sdec, sb.gdec, d);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) r[t] = __fmul_rn(r[t], inv);
-            *reinterpret_cast<uint32_t*>(a.rs_codes + row * (K / 2) + (int64_t)c * 4) = cvt_e2m1x8(r);
-            uint32_t word = gather4(er, lane, 2);
-            if ((lane & 7) == 0)
-                *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, c / 2, nsf)) = word;
+            for (int t = 0; t < 8; ++t) y[8 + t] = __fsub_rn(y[8 + t], d[t]);   // y := r
+            const uint32_t er = cvt_e4m3(__fmul_rn(amaxE<16>(y), sr.k1));
+            const float inv = s_inv[er];
+            float t8[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[t], inv);
+            const uint32_t c0 = cvt_e2m1x8(t8);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[8 + t], inv);
+            const uint32_t c1 = cvt_e2m1x8(t8);
+            *reinterpret_cast<uint2*>(a.rs_codes + row * (K / 2) + (int64_t)cb * 8) = make_uint2(c0, c1);
+            a.rs_scales[sf_off(row, cb, nsf)] = (uint8_t)er;
+            cur = nxt;
+            lb = ln;
+            bc = nbc;
+            bs = nbs;
         }
     }
 }
 
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
-    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT>;
+    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24>;
     static int blocks_per_sm = 0;          // same for every device of one architecture
     if (blocks_per_sm == 0) {
         int b = 0;
@@ -385,8 +579,11 @@ cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
         if (e != cudaSuccess) return e;
         blocks_per_sm = b;
     }
+    // Enough warps for one row each in phase 1 and about four 32-block
+    // groups each in phases 2 and 3, capped at what is resident.
     int64_t Mpad = (a.M + 127) / 128 * 128;
-    int64_t want = (Mpad + kWarps - 1) / kWarps;
+    int64_t groups = a.M * (int64_t)(a.K / (FMT == 0 ? 16 : 32)) / 32;
+    int64_t want = std::max((Mpad + kWarps - 1) / kWarps, (groups + 4 * kWarps - 1) / (4 * kWarps));
     int64_t cap = (int64_t)blocks_per_sm * max_blocks;
     int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
     cudaLaunchConfig_t cfg = {};
@@ -398,16 +595,17 @@ cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     attr[0].id = cudaLaunchAttributeCooperative;   // grid barriers: all blocks co-resident
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = (FMT == 0) ? 1 : 0;
+    cfg.numAttrs = (FMT == 0 || HAS_GAMMA) ? 1 : 0;   // any grid barrier needs co-residency
     return cudaLaunchKernelEx(&cfg, kfn, a);
 }
 
 template <int FMT, bool HAS_GAMMA, bool WEIGHT>
 cudaError_t launch_m(const PrepArgs& a, int m, cudaStream_t s, int sms) {
     switch (m) {
-        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT>(a, s, sms);
-        case 4: return launch_one<FMT, HAS_GAMMA, 4, WEIGHT>(a, s, sms);
-        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT>(a, s, sms);
+        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false>(a, s, sms);
+        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true>(a, s, sms)
+                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false>(a, s, sms);
+        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false>(a, s, sms);
     }
 }
 
@@ -438,8 +636,8 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     if (e != cudaSuccess) return e;
     const bool g = p.gamma != nullptr;
     if (p.weight) {
-        return p.fmt == 0 ? launch_one<0, false, 8, true>(a, s, sms)
-                          : launch_one<1, false, 8, true>(a, s, sms);
+        return p.fmt == 0 ? launch_one<0, false, 8, true, false>(a, s, sms)
+                          : launch_one<1, false, 8, true, false>(a, s, sms);
     }
     if (p.fmt == 0) return g ? launch_m<0, true, false>(a, p.m, s, sms) : launch_m<0, false, false>(a, p.m, s, sms);
     return g ? launch_m<1, true, false>(a, p.m, s, sms) : launch_m<1, false, false>(a, p.m, s, sms);
