@@ -21,7 +21,8 @@ from typing import Optional
 __all__ = [
     "NVFP4", "MXFP4", "SharqError", "load_sharq_ops", "scale_bytes",
     "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
-    "prepare", "prepare_noalloc", "linear", "moe_linear", "last_device_status",
+    "prepare", "prepare_noalloc", "linear", "moe_linear", "moe_workspace_bytes",
+    "last_device_status",
 ]
 
 NVFP4, MXFP4 = 0, 1
@@ -85,8 +86,10 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_prepare.restype = I
         L.sharq_linear.argtypes = [ctypes.POINTER(_Prepared), ctypes.POINTER(_Weight), P, I, P]
         L.sharq_linear.restype = I
+        L.sharq_moe_workspace_bytes.argtypes = [I64, I, I, I]
+        L.sharq_moe_workspace_bytes.restype = SZ
         L.sharq_moe_linear.argtypes = [ctypes.POINTER(_Prepared), P, P, I, I64,
-                                       ctypes.POINTER(_Weight), P, I, P]
+                                       ctypes.POINTER(_Weight), P, I, P, SZ, P]
         L.sharq_moe_linear.restype = I
         L.sharq_prepare_noalloc.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P]
         L.sharq_prepare_noalloc.restype = I
@@ -254,20 +257,31 @@ def linear(x: Prepared, w: Weight, out_fp32: bool = False, out=None, stream=None
     return Y
 
 
+def moe_workspace_bytes(T: int, E: int, K: int, fmt="nvfp4") -> int:
+    return int(load_sharq_ops().sharq_moe_workspace_bytes(T, E, K, _fmt(fmt)))
+
+
 def moe_linear(x: Prepared, row_index, offsets, w: Weight, out_fp32: bool = False, out=None,
-               stream=None):
-    """Grouped two-path linear; row_index: int32 [T] device tensor or None,
-    offsets: int32 [E+1] device tensor, w: stacked expert weights."""
+               ws=None, T: Optional[int] = None, stream=None):
+    """Grouped two-path linear.  row_index: int32 [T] device tensor (or None:
+    dispatched row t is prepared row t); offsets: int32 [E+1] device tensor;
+    w: E stacked expert weights (Weight.empty(..., E=E))."""
     import torch
     L = load_sharq_ops()
-    T = int(row_index.numel()) if row_index is not None else x.M
+    if T is None:
+        T = int(row_index.numel()) if row_index is not None else x.M
+    E = int(offsets.numel()) - 1
     dt = torch.float32 if out_fp32 else torch.bfloat16
-    Y = out if out is not None else torch.empty((T, w.N), dtype=dt, device=x.bb_codes.device)
+    dev = x.bb_scales.device
+    Y = out if out is not None else torch.empty((T, w.N), dtype=dt, device=dev)
+    need = moe_workspace_bytes(T, E, x.K, x.fmt)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=dev)
     cx, cw = x._c(), w._c()
     _check("sharq_moe_linear",
-           L.sharq_moe_linear(ctypes.byref(cx), _ptr(row_index), offsets.data_ptr(),
-                              int(offsets.numel()) - 1, T, ctypes.byref(cw), Y.data_ptr(),
-                              1 if out_fp32 else 0, _stream(stream)))
+           L.sharq_moe_linear(ctypes.byref(cx), _ptr(row_index), offsets.data_ptr(), E, T,
+                              ctypes.byref(cw), Y.data_ptr(), 1 if out_fp32 else 0,
+                              ws.data_ptr(), ws.numel(), _stream(stream)))
     return Y
 
 

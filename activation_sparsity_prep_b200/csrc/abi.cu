@@ -141,18 +141,38 @@ sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w, void* 
                                             sharq::device_sm_count()));
 }
 
+size_t sharq_moe_workspace_bytes(int64_t T, int E, int K, int fmt) {
+    if (!valid_fmt(fmt) || !valid_shape(T, K) || E <= 0) return 0;
+    return sharq::moe_ws_bytes(T, E, K, fmt);
+}
+
 sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
                               const int32_t* expert_offsets, int E, int64_t T,
-                              const sharq_weight* w, void* Y, int y_is_fp32, void* stream) {
-    sharq_status st = check_linear_args(x, w, Y);
-    if (st != SHARQ_OK) return st;
+                              const sharq_weight* w, void* Y, int y_is_fp32, void* ws,
+                              size_t ws_bytes, void* stream) {
+    if (!x || !w) return SHARQ_ERR_INVALID_ARG;
     if (!expert_offsets || E <= 0 || T < 0 || (!row_index && T != x->M)) return SHARQ_ERR_INVALID_ARG;
+    if (E > 256) return SHARQ_ERR_UNSUPPORTED;
+    if (T > 0 && (!Y || !ws)) return SHARQ_ERR_INVALID_ARG;
+    if (!valid_fmt(x->fmt) || x->fmt != w->fmt || !valid_shape(x->M, x->K) || x->K != w->K)
+        return SHARQ_ERR_INVALID_ARG;
+    if (w->N <= 0 || w->N % 128 != 0 || !w->codes || !w->scales || !w->tensor_scale)
+        return SHARQ_ERR_INVALID_ARG;
+    if (!x->bb_tscale || !x->rs_tscale) return SHARQ_ERR_INVALID_ARG;
+    if (x->M > 0 && (!x->bb_codes || !x->bb_scales || !x->rs_codes || !x->rs_scales))
+        return SHARQ_ERR_INVALID_ARG;
+    if (!aligned16(x->bb_codes) || !aligned16(x->bb_scales) || !aligned16(x->rs_codes) ||
+        !aligned16(x->rs_scales) || !aligned16(w->codes) || !aligned16(w->scales) || !aligned16(Y) ||
+        !aligned16(ws) || ((uintptr_t)row_index & 3u) || ((uintptr_t)expert_offsets & 3u))
+        return SHARQ_ERR_INVALID_ARG;
+    if (ws_bytes < sharq::moe_ws_bytes(T, E, x->K, x->fmt)) return SHARQ_ERR_INVALID_ARG;
+    if (T == 0) return SHARQ_OK;
     sharq::LinearLaunch p{};
     p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
     p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
     p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
     p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
-    p.row_index = row_index; p.offsets = expert_offsets; p.E = E; p.T = T;
+    p.row_index = row_index; p.offsets = expert_offsets; p.E = E; p.T = T; p.ws = ws;
     return cuda_status(sharq::launch_moe_linear(p, static_cast<cudaStream_t>(stream),
                                                 sharq::device_sm_count()));
 }

@@ -15,7 +15,8 @@
 //
 // CTA layout (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
 // and MMA issuer, warps 2..5 = epilogue (one TMEM lane quarter each).
-// Tile 128 x 128 x 256 (K in elements), 4-stage mbarrier pipeline.
+// Tile 128 x 128 x 256 (K in elements), 4-stage mbarrier pipeline; one
+// persistent CTA per SM walks the output tiles.
 #include "common.cuh"
 #include "sharq_internal.h"
 
@@ -48,7 +49,8 @@ struct Cfg {
 struct alignas(8) Barriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t acc_full;
+    uint64_t acc_full;      // MMAs of the current tile done (tcgen05.commit)
+    uint64_t acc_empty;     // epilogue has drained the accumulators (4 warps)
     uint32_t tmem_base;
 };
 
@@ -75,31 +77,147 @@ struct EpiArgs {
     int y_fp32;
 };
 
+// One output tile of the (plain or grouped) problem.
+struct TileInfo {
+    int64_t a_row;     // first row of the activation tiles (multiple of 128)
+    int64_t w_row;     // first row of the weight tile in the (stacked) weight
+    int64_t w_sf;      // byte offset of the weight tile's first scale atom
+    int64_t y_row;     // first output row
+    int rows;          // valid output rows in this tile (<= 128)
+    int col;           // first output column
+    int e;             // expert (0 for the plain linear)
+};
+
+constexpr int kMaxExperts = 256;    // keeps the scheduler's shared memory at 3 KiB
+
+// Tile scheduler.  Plain linear: m fastest, so the CTAs working at one time
+// share weight tiles (each weight tile is read from HBM about once) while
+// the activation tiles stay resident in L2.  Grouped linear: expert-major,
+// then n, then m, so one expert's weight and activation rows stay hot in L2
+// while its tiles run; rows of expert e sit at a 128-aligned padded offset
+// of the gathered operands.
+struct Sched {
+    int mt_count, nt_count;    // plain: m-tiles, n-tiles
+    int64_t M;
+    int nsf;                   // scales per row
+    int grouped;
+    const int32_t* offsets;    // grouped: dispatch offsets [E+1] (device)
+    int E;
+    int64_t w_sf_stride;       // grouped: bytes of one expert's scale buffer
+    int N;
+};
+
+struct SchedSmem {
+    int off[kMaxExperts + 1];    // dispatch offsets
+    int poff[kMaxExperts + 1];   // padded row offsets (128-aligned)
+    int tpre[kMaxExperts + 1];   // tile prefix
+};
+
+__device__ __forceinline__ int ceil128(int x) { return (x + 127) >> 7; }
+
+// Exclusive prefix sums of the per-expert padded rows and tiles, by warp 0.
+__device__ void sched_prepare(const Sched& sc, SchedSmem* sm) {
+    if (!sc.grouped) return;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x < 32) {
+        int carry_p = 0, carry_t = 0;
+        for (int base = 0; base < sc.E; base += 32) {
+            const int e = base + lane;
+            int cnt = 0;
+            if (e < sc.E) {
+                const int o0 = sc.offsets[e], o1 = sc.offsets[e + 1];
+                sm->off[e] = o0;
+                cnt = o1 - o0;
+            }
+            int pr = ceil128(cnt) * 128, tl = ceil128(cnt) * sc.nt_count;
+            int ip = pr, it = tl;                      // inclusive warp scans
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int vp = __shfl_up_sync(0xffffffffu, ip, o), vt = __shfl_up_sync(0xffffffffu, it, o);
+                if (lane >= o) { ip += vp; it += vt; }
+            }
+            if (e < sc.E) { sm->poff[e] = carry_p + ip - pr; sm->tpre[e] = carry_t + it - tl; }
+            carry_p += __shfl_sync(0xffffffffu, ip, 31);
+            carry_t += __shfl_sync(0xffffffffu, it, 31);
+        }
+        if (lane == 0) {
+            sm->off[sc.E] = sc.offsets[sc.E];
+            sm->poff[sc.E] = carry_p;
+            sm->tpre[sc.E] = carry_t;
+        }
+    }
+}
+
+__device__ __forceinline__ int sched_count(const Sched& sc, const SchedSmem* sm) {
+    return sc.grouped ? sm->tpre[sc.E] : sc.mt_count * sc.nt_count;
+}
+
+__device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem* sm, int t) {
+    TileInfo ti;
+    if (!sc.grouped) {
+        const int nt = t / sc.mt_count, mt = t - nt * sc.mt_count;
+        ti.a_row = (int64_t)mt * 128;
+        ti.w_row = (int64_t)nt * 128;
+        ti.w_sf = (int64_t)nt * (sc.nsf / 4) * 512;
+        ti.y_row = ti.a_row;
+        ti.rows = (int)(sc.M - ti.a_row < 128 ? sc.M - ti.a_row : 128);
+        ti.col = nt * 128;
+        ti.e = 0;
+        return ti;
+    }
+    int lo = 0, hi = sc.E;                          // largest e with tpre[e] <= t
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (sm->tpre[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int cnt = sm->off[e + 1] - sm->off[e];
+    const int mtn = ceil128(cnt);
+    const int local = t - sm->tpre[e];
+    const int nt = local / mtn, mt = local - nt * mtn;
+    ti.a_row = sm->poff[e] + (int64_t)mt * 128;
+    ti.w_row = (int64_t)e * sc.N + (int64_t)nt * 128;
+    ti.w_sf = (int64_t)e * sc.w_sf_stride + (int64_t)nt * (sc.nsf / 4) * 512;
+    ti.y_row = sm->off[e] + (int64_t)mt * 128;
+    ti.rows = min(128, cnt - mt * 128);
+    ti.col = nt * 128;
+    ti.e = e;
+    return ti;
+}
+
+// Persistent kernel: CTA c computes tiles c, c + G, c + 2G, ...  The TMA
+// producer runs ahead across tile boundaries through a kStages ring; the MMA
+// thread waits only until the epilogue has copied the previous tile's two
+// accumulators out of tensor memory, so the epilogue's global stores overlap
+// the next tile's MMAs.
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_r,
               const __grid_constant__ CUtensorMap tm_w, const uint8_t* __restrict__ sf_b,
               const uint8_t* __restrict__ sf_r, const uint8_t* __restrict__ sf_w, int K,
-              EpiArgs ep) {
+              EpiArgs ep, Sched sc) {
     using C = Cfg<FMT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Barriers* bars = reinterpret_cast<Barriers*>(smem + kStages * C::kStageStride);
+    SchedSmem* ssm = reinterpret_cast<SchedSmem*>(reinterpret_cast<uint8_t*>(bars) + sizeof(Barriers));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mt = blockIdx.x, nt = blockIdx.y;
     const int nk = K / BK;
     const int nsf = K / C::BS;
+    sched_prepare(sc, ssm);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
         mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->acc_empty, 4);
         fence_barrier_init();
     }
     if (warp == 1) { tmem_alloc(&bars->tmem_base, kTmemCols); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const int ntiles = sched_count(sc, ssm);
     const uint32_t tmem = bars->tmem_base;
     const uint32_t t_acc_b = tmem, t_acc_r = tmem + BN;
     const uint32_t t_sfa_b = tmem + 2 * BN;
@@ -109,77 +227,94 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     if (warp == 0) {
         if (lane == 0) {
             prefetch_tmap(&tm_b); prefetch_tmap(&tm_r); prefetch_tmap(&tm_w);
-            const uint8_t* gb = sf_b + (int64_t)mt * (nsf / 4) * 512;
-            const uint8_t* gr = sf_r + (int64_t)mt * (nsf / 4) * 512;
-            const uint8_t* gw = sf_w + (int64_t)nt * (nsf / 4) * 512;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kStages;
-                if (kb >= kStages && !mbar_wait(&bars->empty[s], ((kb / kStages) - 1) & 1)) break;
-                uint8_t* st = smem + s * C::kStageStride;
-                mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
-                tma_load_2d(st, &tm_b, &bars->full[s], kb * (BK / 2), mt * BM);
-                tma_load_2d(st + kTileBytes, &tm_r, &bars->full[s], kb * (BK / 2), mt * BM);
-                tma_load_2d(st + 2 * kTileBytes, &tm_w, &bars->full[s], kb * (BK / 2), nt * BN);
-                const int64_t sfo = (int64_t)kb * C::kAtoms * 512;
-                bulk_load(st + 3 * kTileBytes, gb + sfo, C::kSfBytes, &bars->full[s]);
-                bulk_load(st + 3 * kTileBytes + C::kSfBytes, gr + sfo, C::kSfBytes, &bars->full[s]);
-                bulk_load(st + 3 * kTileBytes + 2 * C::kSfBytes, gw + sfo, C::kSfBytes, &bars->full[s]);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const TileInfo ti = sched_tile(sc, ssm, tile);
+                const uint8_t* gb = sf_b + (ti.a_row >> 7) * (nsf / 4) * 512;
+                const uint8_t* gr = sf_r + (ti.a_row >> 7) * (nsf / 4) * 512;
+                const uint8_t* gw = sf_w + ti.w_sf;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t s = it % kStages;
+                    if (it >= kStages && !mbar_wait(&bars->empty[s], ((it / kStages) - 1) & 1)) { ok = false; break; }
+                    uint8_t* st = smem + s * C::kStageStride;
+                    mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
+                    tma_load_2d(st, &tm_b, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                    tma_load_2d(st + kTileBytes, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                    tma_load_2d(st + 2 * kTileBytes, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
+                    const int64_t sfo = (int64_t)kb * C::kAtoms * 512;
+                    bulk_load(st + 3 * kTileBytes, gb + sfo, C::kSfBytes, &bars->full[s]);
+                    bulk_load(st + 3 * kTileBytes + C::kSfBytes, gr + sfo, C::kSfBytes, &bars->full[s]);
+                    bulk_load(st + 3 * kTileBytes + 2 * C::kSfBytes, gw + sfo, C::kSfBytes, &bars->full[s]);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            uint32_t it = 0, tc = 0;
             bool ok = true;
-            for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % kStages;
-                if (!mbar_wait(&bars->full[s], (kb / kStages) & 1)) { ok = false; break; }
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+                // the epilogue must have drained the previous tile's accumulators
+                if (tc > 0 && !mbar_wait(&bars->acc_empty, (tc - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
-                uint8_t* st = smem + s * C::kStageStride;
-                const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + kTileBytes);
-                const uint32_t a_w = smem_u32(st + 2 * kTileBytes);
-                const uint32_t s_b = smem_u32(st + 3 * kTileBytes);
-                const uint32_t s_r = s_b + C::kSfBytes, s_w = s_b + 2 * C::kSfBytes;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t s = it % kStages;
+                    if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    uint8_t* st = smem + s * C::kStageStride;
+                    const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + kTileBytes);
+                    const uint32_t a_w = smem_u32(st + 2 * kTileBytes);
+                    const uint32_t s_b = smem_u32(st + 3 * kTileBytes);
+                    const uint32_t s_r = s_b + C::kSfBytes, s_w = s_b + 2 * C::kSfBytes;
 #pragma unroll
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    tc_cp_32x128b_warpx4(t_sfa_b + 4 * at, sdesc_sf_atom(s_b + 512 * at));
-                    tc_cp_32x128b_warpx4(t_sfa_r + 4 * at, sdesc_sf_atom(s_r + 512 * at));
-                    tc_cp_32x128b_warpx4(t_sfb + 4 * at, sdesc_sf_atom(s_w + 512 * at));
-                }
+                    for (int at = 0; at < C::kAtoms; ++at) {
+                        tc_cp_32x128b_warpx4(t_sfa_b + 4 * at, sdesc_sf_atom(s_b + 512 * at));
+                        tc_cp_32x128b_warpx4(t_sfa_r + 4 * at, sdesc_sf_atom(s_r + 512 * at));
+                        tc_cp_32x128b_warpx4(t_sfb + 4 * at, sdesc_sf_atom(s_w + 512 * at));
+                    }
 #pragma unroll
-                for (int j = 0; j < BK / 64; ++j) {
-                    const int at = j / C::kStepsPerAtom;
-                    const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
-                    const uint32_t col = 4 * at;
-                    const uint64_t db = sdesc_sw128(a_w + 32 * j);
-                    const uint32_t acc = (kb | j) ? 1u : 0u;
-                    mma<FMT>(t_acc_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + col,
-                             acc, sf_id);
-                    mma<FMT>(t_acc_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + col,
-                             acc, sf_id);
+                    for (int j = 0; j < BK / 64; ++j) {
+                        const int at = j / C::kStepsPerAtom;
+                        const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
+                        const uint32_t col = 4 * at;
+                        const uint64_t db = sdesc_sw128(a_w + 32 * j);
+                        const uint32_t acc = (kb | j) ? 1u : 0u;
+                        mma<FMT>(t_acc_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + col,
+                                 acc, sf_id);
+                        mma<FMT>(t_acc_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + col,
+                                 acc, sf_id);
+                    }
+                    tc_commit(&bars->empty[s]);
                 }
-                tc_commit(&bars->empty[s]);
+                tc_commit(&bars->acc_full);
             }
-            tc_commit(&bars->acc_full);
         }
     } else {
         // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = rows of the tile.
         const int q = warp & 3;
-        const int64_t row = (int64_t)mt * BM + q * 32 + lane;
-        const bool ok = mbar_wait(&bars->acc_full, 0);
-        tc_fence_after();
-        if (ok) {
-            const float gw = *ep.w_tscale;
-            const float gb = *ep.bb_tscale * gw, gr = *ep.rs_tscale * gw;
-            const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const float gbb = *ep.bb_tscale, grr = *ep.rs_tscale;
+        uint32_t tc = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+            const TileInfo ti = sched_tile(sc, ssm, tile);
+            const float gwv = ep.w_tscale[ti.e];
+            const float gb = gbb * gwv, gr = grr * gwv;
+            const int r_local = q * 32 + lane;
+            const int64_t row = ti.y_row + r_local;
+            const bool row_ok = r_local < ti.rows;
+            const bool ok = mbar_wait(&bars->acc_full, tc & 1);
+            tc_fence_after();
+            if (!ok) break;
+            const int64_t col0 = ti.col;
+            if (ep.y_fp32) {
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t vb[32], vr[32];
-                tmem_ld_32x32b_x32(t_acc_b + lane_off + cc * 32, vb);
-                tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
-                tmem_ld_wait();
-                if (row < ep.M) {
-                    const int64_t col0 = (int64_t)nt * BN + cc * 32;
-                    if (ep.y_fp32) {
-                        float* y = static_cast<float*>(ep.Y) + row * ep.N + col0;
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    uint32_t vb[32], vr[32];
+                    tmem_ld_32x32b_x32(t_acc_b + lane_off + cc * 32, vb);
+                    tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float* y = static_cast<float*>(ep.Y) + row * ep.N + col0 + cc * 32;
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {
                             float4 o;
@@ -189,21 +324,38 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                             o.w = gb * __uint_as_float(vb[i + 3]) + gr * __uint_as_float(vr[i + 3]);
                             *reinterpret_cast<float4*>(y + i) = o;
                         }
-                    } else {
-                        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(ep.Y) + row * ep.N + col0;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                float lo = gb * __uint_as_float(vb[i + 2 * h]) + gr * __uint_as_float(vr[i + 2 * h]);
-                                float hi = gb * __uint_as_float(vb[i + 2 * h + 1]) + gr * __uint_as_float(vr[i + 2 * h + 1]);
-                                __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
-                                w[h] = *reinterpret_cast<uint32_t*>(&p);
-                            }
-                            *reinterpret_cast<uint4*>(y + i) = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
                     }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->acc_empty);
+            } else {
+                // drain both accumulators into 64 packed bf16x2 registers, hand
+                // the tensor memory back, then store
+                uint32_t out[BN / 2];
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    uint32_t vb[32], vr[32];
+                    tmem_ld_32x32b_x32(t_acc_b + lane_off + cc * 32, vb);
+                    tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) {
+                        float lo = gb * __uint_as_float(vb[2 * h]) + gr * __uint_as_float(vr[2 * h]);
+                        float hi = gb * __uint_as_float(vb[2 * h + 1]) + gr * __uint_as_float(vr[2 * h + 1]);
+                        __nv_bfloat162 p2 = __floats2bfloat162_rn(lo, hi);
+                        out[cc * 16 + h] = *reinterpret_cast<uint32_t*>(&p2);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->acc_empty);
+                if (row_ok) {
+                    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(ep.Y) + row * ep.N + col0;
+#pragma unroll
+                    for (int i = 0; i < BN / 8; ++i)
+                        *reinterpret_cast<uint4*>(y + 8 * i) =
+                            make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
                 }
             }
         }
@@ -247,42 +399,153 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_b
 }
 
 template <int FMT>
-cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s) {
-    using C = Cfg<FMT>;
-    CUtensorMap tb, tr, tw;
-    if (!make_code_map(&tb, p.bb_codes, p.M, p.K / 2, BM) ||
-        !make_code_map(&tr, p.rs_codes, p.M, p.K / 2, BM) ||
-        !make_code_map(&tw, p.w_codes, p.N, p.K / 2, BN))
-        return cudaErrorInvalidValue;
-    const size_t smem = kStages * C::kStageStride + sizeof(Barriers) + 1024;
-    auto kfn = linear_kernel<FMT>;
+size_t linear_smem_bytes() {
+    return kStages * Cfg<FMT>::kStageStride + sizeof(Barriers) + sizeof(SchedSmem) + 1024;
+}
+
+template <int FMT>
+cudaError_t ensure_smem_attr() {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(linear_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)linear_smem_bytes<FMT>());
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_set[dev] = true;
     }
+    return cudaSuccess;
+}
+
+// A_rows: rows of the activation operands (gathered and padded for the
+// grouped form); W_rows: rows of the (stacked) weight.
+template <int FMT>
+cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void* rs_codes,
+                        const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
+                        const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
+    CUtensorMap tb, tr, tw;
+    if (!make_code_map(&tb, bb_codes, A_rows, p.K / 2, BM) ||
+        !make_code_map(&tr, rs_codes, A_rows, p.K / 2, BM) ||
+        !make_code_map(&tw, p.w_codes, W_rows, p.K / 2, BN))
+        return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem_attr<FMT>();
+    if (e != cudaSuccess) return e;
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
-    dim3 grid((unsigned)((p.M + BM - 1) / BM), (unsigned)(p.N / BN));
-    kfn<<<grid, kThreads, smem, s>>>(tb, tr, tw, static_cast<const uint8_t*>(p.bb_scales),
-                                     static_cast<const uint8_t*>(p.rs_scales),
-                                     static_cast<const uint8_t*>(p.w_scales), p.K, ep);
+    const int grid = std::max(1, std::min(max_tiles, std::max(1, sms)));
+    linear_kernel<FMT><<<grid, kThreads, linear_smem_bytes<FMT>(), s>>>(
+        tb, tr, tw, static_cast<const uint8_t*>(bb_scales), static_cast<const uint8_t*>(rs_scales),
+        static_cast<const uint8_t*>(p.w_scales), p.K, ep, sc);
     return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
+    Sched sc{};
+    sc.mt_count = (int)((p.M + BM - 1) / BM);
+    sc.nt_count = p.N / BN;
+    sc.M = p.M;
+    sc.nsf = p.K / Cfg<FMT>::BS;
+    sc.grouped = 0;
+    sc.N = p.N;
+    return launch_gemm<FMT>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p, p.N, sc,
+                            sc.mt_count * sc.nt_count, s, sms);
+}
+
+// ------------------------------------------------------------ grouped ----
+// Gather: dispatched row t of expert e (offsets[e] <= t < offsets[e+1])
+// reads prepared row row_index[t] (or t) and is written to padded row
+// poff[e] + (t - offsets[e]) of the workspace operands: both code rows and
+// both rows of scale atoms (4-byte words of four scales).
+template <int FMT>
+__global__ void __launch_bounds__(256)
+moe_gather_kernel(const uint8_t* __restrict__ bb_codes, const uint8_t* __restrict__ bb_scales,
+                  const uint8_t* __restrict__ rs_codes, const uint8_t* __restrict__ rs_scales,
+                  const int32_t* __restrict__ row_index, Sched sc, int K, int64_t T,
+                  uint8_t* __restrict__ gb_codes, uint8_t* __restrict__ gb_scales,
+                  uint8_t* __restrict__ gr_codes, uint8_t* __restrict__ gr_scales) {
+    __shared__ SchedSmem ssm;
+    sched_prepare(sc, &ssm);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * 8;
+    const int row_bytes = K / 2;
+    const int words = sc.nsf / 4;
+    for (int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += warps) {
+        int lo = 0, hi = sc.E;                      // expert of row t
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (ssm.off[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int64_t src = row_index ? (int64_t)row_index[t] : t;
+        const int64_t dst = ssm.poff[lo] + (t - ssm.off[lo]);
+        const uint4* sb = reinterpret_cast<const uint4*>(bb_codes + src * row_bytes);
+        const uint4* sr = reinterpret_cast<const uint4*>(rs_codes + src * row_bytes);
+        uint4* db = reinterpret_cast<uint4*>(gb_codes + dst * row_bytes);
+        uint4* dr = reinterpret_cast<uint4*>(gr_codes + dst * row_bytes);
+        for (int i = lane; i < row_bytes / 16; i += 32) { db[i] = sb[i]; dr[i] = sr[i]; }
+        const int64_t so = (src >> 7) * words * 512 + (src & 31) * 16 + ((src >> 5) & 3) * 4;
+        const int64_t d0 = (dst >> 7) * words * 512 + (dst & 31) * 16 + ((dst >> 5) & 3) * 4;
+        for (int w = lane; w < words; w += 32) {
+            *reinterpret_cast<uint32_t*>(gb_scales + d0 + w * 512) =
+                *reinterpret_cast<const uint32_t*>(bb_scales + so + w * 512);
+            *reinterpret_cast<uint32_t*>(gr_scales + d0 + w * 512) =
+                *reinterpret_cast<const uint32_t*>(rs_scales + so + w * 512);
+        }
+    }
+}
+
+template <int FMT>
+cudaError_t launch_moe_t(const LinearLaunch& p, cudaStream_t s, int sms) {
+    constexpr int BS = Cfg<FMT>::BS;
+    const int nsf = p.K / BS;
+    const int64_t rows_max = moe_padded_rows(p.T, p.E);
+    uint8_t* ws = static_cast<uint8_t*>(p.ws);
+    uint8_t* gb_codes = ws;
+    uint8_t* gr_codes = gb_codes + rows_max * (p.K / 2);
+    uint8_t* gb_scales = gr_codes + rows_max * (p.K / 2);
+    uint8_t* gr_scales = gb_scales + rows_max * nsf;
+    Sched sc{};
+    sc.nt_count = p.N / BN;
+    sc.M = p.T;
+    sc.nsf = nsf;
+    sc.grouped = 1;
+    sc.offsets = p.offsets;
+    sc.E = p.E;
+    sc.w_sf_stride = (int64_t)((p.N + 127) / 128 * 128) * nsf;
+    sc.N = p.N;
+    if (p.T > 0) {
+        const int gblocks = (int)std::min<int64_t>((p.T + 7) / 8, (int64_t)sms * 8);
+        moe_gather_kernel<FMT><<<std::max(1, gblocks), 256, 0, s>>>(
+            static_cast<const uint8_t*>(p.bb_codes), static_cast<const uint8_t*>(p.bb_scales),
+            static_cast<const uint8_t*>(p.rs_codes), static_cast<const uint8_t*>(p.rs_scales),
+            p.row_index, sc, p.K, p.T, gb_codes, gb_scales, gr_codes, gr_scales);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const int max_tiles = (int)((p.T + 127) / 128 + p.E) * sc.nt_count;
+    LinearLaunch q = p;
+    q.M = p.T;
+    return launch_gemm<FMT>(gb_codes, gb_scales, gr_codes, gr_scales, rows_max, q,
+                            (int64_t)p.E * p.N, sc, max_tiles, s, sms);
 }
 
 }  // namespace
 
 unsigned take_status_linear() { return take_tu_status(); }
 
-cudaError_t launch_linear(const LinearLaunch& p, cudaStream_t s, int /*sms*/) {
+cudaError_t launch_linear(const LinearLaunch& p, cudaStream_t s, int sms) {
     if (p.M == 0) return cudaSuccess;
-    return p.fmt == 0 ? launch_linear_t<0>(p, s) : launch_linear_t<1>(p, s);
+    return p.fmt == 0 ? launch_linear_t<0>(p, s, sms) : launch_linear_t<1>(p, s, sms);
 }
 
-cudaError_t launch_moe_linear(const LinearLaunch&, cudaStream_t, int) {
-    return cudaErrorNotSupported;
+cudaError_t launch_moe_linear(const LinearLaunch& p, cudaStream_t s, int sms) {
+    if (p.E > kMaxExperts) return cudaErrorNotSupported;
+    return p.fmt == 0 ? launch_moe_t<0>(p, s, sms) : launch_moe_t<1>(p, s, sms);
+}
+
+size_t moe_ws_bytes(int64_t T, int E, int K, int fmt) {
+    const int nsf = K / (fmt == 0 ? 16 : 32);
+    return (size_t)moe_padded_rows(T, E) * (size_t)(K + 2 * nsf);
 }
 
 }  // namespace sharq

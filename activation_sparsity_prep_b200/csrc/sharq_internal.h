@@ -49,7 +49,12 @@ struct LinearLaunch {
     const int32_t* offsets;   // null for the plain linear
     int E;
     int64_t T;
+    void* ws;                 // grouped form: gathered operands
 };
+
+// Rows of the gathered, per-expert 128-aligned activation operands.
+inline int64_t moe_padded_rows(int64_t T, int E) { return (T + 128 * (int64_t)E + 127) / 128 * 128; }
+size_t moe_ws_bytes(int64_t T, int E, int K, int fmt);
 
 cudaError_t launch_linear(const LinearLaunch& p, cudaStream_t s, int sms);
 cudaError_t launch_moe_linear(const LinearLaunch& p, cudaStream_t s, int sms);

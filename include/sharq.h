@@ -144,17 +144,26 @@ SHARQ_API sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16,
 SHARQ_API sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w,
                           void* Y, int y_is_fp32, void* stream);
 
-/* Grouped (mixture-of-experts) form of sharq_linear: dispatched row t
- * (0 <= t < T) reads prepared row row_index[t] (row_index NULL: row t) and is
- * multiplied by expert e's weight when offsets[e] <= t < offsets[e+1].
- * expert_offsets is a DEVICE int32 array [E+1] with offsets[0] = 0 and
- * offsets[E] = T, non-decreasing.  w holds E stacked weights (see
- * sharq_weight).  The activation tensor scales are those of the whole
- * prepare call.  Y is [T, N]. */
+/* Grouped (mixture-of-experts) form of sharq_linear (the pages evaluate the
+ * method on a mixture-of-experts model; each expert is a SharQ linear):
+ * dispatched row t (0 <= t < T) reads prepared row row_index[t] (row_index
+ * NULL: row t, which needs T == x->M) and is multiplied by expert e's
+ * weight when offsets[e] <= t < offsets[e+1]:
+ *   Y[t,j] = G_w[e] * (G_b * S_b[t,j] + G_r * S_r[t,j]).
+ * expert_offsets is a DEVICE int32 array [E+1], offsets[0] = 0, offsets[E]
+ * = T, non-decreasing; row_index is a DEVICE int32 array [T] of rows < x->M.
+ * w holds E stacked weights (see sharq_weight), 1 <= E <= 256.  The
+ * activation tensor scales are those of the whole prepare call.  Y is [T, N]
+ * in dispatch order.  The call first gathers each expert's rows into ws
+ * (sharq_moe_workspace_bytes(T, E, K, fmt) bytes, caller-owned, content on
+ * entry irrelevant), padded to 128-row groups, then runs one persistent
+ * grouped GEMM over all experts. */
+SHARQ_API size_t sharq_moe_workspace_bytes(int64_t T, int E, int K, int fmt);
+
 SHARQ_API sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
-                              const int32_t* expert_offsets, int E, int64_t T,
-                              const sharq_weight* w, void* Y, int y_is_fp32,
-                              void* stream);
+                                        const int32_t* expert_offsets, int E, int64_t T,
+                                        const sharq_weight* w, void* Y, int y_is_fp32,
+                                        void* ws, size_t ws_bytes, void* stream);
 
 /* Largest M that sharq_prepare_noalloc() accepts (its fixed scratch array
  * holds 64 bytes plus 4 bytes per row: 1 MiB + 64 bytes in all). */

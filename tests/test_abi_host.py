@@ -73,8 +73,16 @@ def test_linear_rejects_mismatched_operands():
     assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0, None) == 1
     w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 0)
     assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1008, 0, None) == 1   # misaligned Y
-    assert L.sharq_moe_linear(ctypes.byref(cp), None, None, 4, 16, ctypes.byref(w), 0x1000, 0, None) == 1
-    assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 4, 17, ctypes.byref(w), 0x1000, 0, None) == 1
+    ws = sq.moe_workspace_bytes(16, 4, 256)
+    assert ws >= (16 + 4 * 128) * (256 + 32)
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, None, 4, 16, ctypes.byref(w), 0x1000, 0,
+                              0x1000, ws, None) == 1                       # no offsets
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 4, 17, ctypes.byref(w), 0x1000, 0,
+                              0x1000, ws, None) == 1                       # T != M without row_index
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000, 0,
+                              0x1000, ws - 1, None) == 1                   # workspace too small
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 300, 16, ctypes.byref(w), 0x1000, 0,
+                              0x1000, 1 << 30, None) == 2                  # too many experts
 
 
 def test_status_strings():
