@@ -49,8 +49,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
     ap.add_argument("--workload", default="llama8b")
-    ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--M", type=int, default=None,
+                    help="rows per linear (default: 2048 for llama8b, the workload's own M otherwise)")
     ap.add_argument("--fmt", default="nvfp4")
+    ap.add_argument("--nm", default="2:4", help="n:m of the backbone mask")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -244,6 +246,72 @@ def run_reference(args):
 
 # ------------------------------------------------------------ GPU arm ----
 
+def nm_of(args):
+    n, m = (int(v) for v in args.nm.split(":"))
+    return n, m
+
+
+def build_units(args, dev):
+    """Device buffers and closures for one step of the chosen workload.
+    A unit is one prepare followed by one (plain or grouped) linear."""
+    import torch
+
+    import activation_sparsity_prep_b200 as sq
+
+    W = wl.WORKLOADS[args.workload]
+    fmt = sq._FMT[args.fmt]
+    n, m = nm_of(args)
+    bf = torch.bfloat16
+    up = lambda a: torch.from_numpy(a).view(bf).to(dev)
+    units = []
+    if W.moe is None:
+        M = args.M
+        for L in W.linears:
+            d = wl.linear_inputs(W, L, M)
+            X, g = up(d["X"]), (None if d["gamma"] is None else up(d["gamma"]))
+            Wt = up(d["W"])
+            w = sq.quantize_weight(Wt, fmt)
+            del Wt
+            P = sq.Prepared.empty(M, L.K, n, m, fmt, device=dev)
+            ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
+            Y = torch.empty((M, L.N), dtype=bf, device=dev)
+            u = dict(name=L.name, rows=M, prep_rows=M, N=L.N, K=L.K, X=X, Y=Y)
+            u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
+            u["gemm"] = (lambda P=P, w=w, Y=Y: sq.linear(P, w, out=Y))
+            units.append(u)
+        desc = (f"{W.name}: " + ", ".join(f"{L.name} {L.K}x{L.N}" for L in W.linears)
+                + f"; M={M}, prepare+linear each")
+        return units, desc, M
+    T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
+    ri, off = wl.group_by_expert(wl.routing(W.cfg, T, E, topk), E)
+    ri_d = torch.from_numpy(ri).to(dev)
+    off_d = torch.from_numpy(off).to(dev)
+    for li, L in enumerate(W.linears):
+        rows_in = T if li == 0 else T * topk             # gate_up reads tokens, down dispatched rows
+        X = up(wl.activation(W.dist, W.cfg, L.index, rows_in, L.K))
+        g = up(wl.gamma_ones(L.K)) if L.norm else None
+        w = sq.Weight.empty(L.N, L.K, fmt, device=dev, E=E)
+        sb = sq.scale_bytes(L.N, L.K, fmt)
+        for e in range(E):
+            we = sq.Weight(w.codes[e], w.scales[e * sb:(e + 1) * sb], w.tensor_scale[e:e + 1],
+                           L.N, L.K, w.fmt)
+            sq.quantize_weight(up(wl.weight(W.cfg * 1000 + li, 100 + e, L.N, L.K)), fmt, out=we)
+        P = sq.Prepared.empty(rows_in, L.K, n, m, fmt, device=dev)
+        ws = torch.empty(max(256, sq.prepare_workspace_bytes(rows_in, L.K, fmt)), dtype=torch.uint8, device=dev)
+        mws = torch.empty(sq.moe_workspace_bytes(T * topk, E, L.K, fmt), dtype=torch.uint8, device=dev)
+        Y = torch.empty((T * topk, L.N), dtype=bf, device=dev)
+        rix = ri_d if li == 0 else None
+        u = dict(name=L.name, rows=T * topk, prep_rows=rows_in, N=L.N, K=L.K, X=X, Y=Y)
+        u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
+        u["gemm"] = (lambda P=P, w=w, Y=Y, rix=rix, mws=mws:
+                     sq.moe_linear(P, rix, off_d, w, out=Y, ws=mws, T=T * topk))
+        units.append(u)
+    desc = (f"{W.name}: Qwen3-30B-A3B-shaped expert layer, {T} tokens, {E} experts, top-{topk}; "
+            f"gate_up {W.linears[0].K}x{W.linears[0].N} (rows gathered by index), "
+            f"down {W.linears[1].K}x{W.linears[1].N} (rows in dispatch order); grouped prepare+linear")
+    return units, desc, T
+
+
 def run_sharq(args):
     import torch
     import torch.distributed as dist
@@ -256,46 +324,31 @@ def run_sharq(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local)
-    W = wl.WORKLOADS[args.workload]
-    M = args.M
     fmt = sq._FMT[args.fmt]
-    linears = make_inputs(W, M)
-
-    # device buffers
-    bufs = []
-    for L, d in linears:
-        X = torch.from_numpy(d["X"]).view(torch.bfloat16).to(dev)
-        g = None if d["gamma"] is None else torch.from_numpy(d["gamma"]).view(torch.bfloat16).to(dev)
-        Wt = torch.from_numpy(d["W"]).view(torch.bfloat16).to(dev)
-        w = sq.quantize_weight(Wt, fmt)
-        del Wt
-        P = sq.Prepared.empty(M, L.K, 2, 4, fmt, device=dev)
-        ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
-        Y = torch.empty((M, L.N), dtype=torch.bfloat16, device=dev)
-        bufs.append(dict(L=L, X=X, g=g, w=w, P=P, ws=ws, Y=Y))
+    n, m = nm_of(args)
+    units, desc, tokens_per_step = build_units(args, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def step():
-        for b in bufs:
-            sq.prepare(b["X"], b["g"], wl.EPS, 2, 4, fmt, out=b["P"], ws=b["ws"])
-            sq.linear(b["P"], b["w"], out=b["Y"])
+        for u in units:
+            u["prep"]()
+            u["gemm"]()
 
     # eager warm-up (lazy init), then capture one step with per-kernel events
     step()
     torch.cuda.synchronize()
     assert sq.last_device_status() == 0
-    nev = 2 * len(bufs) + 1
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)]
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(units) + 1)]
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
             evs[0].record()
-            for i, b in enumerate(bufs):
-                sq.prepare(b["X"], b["g"], wl.EPS, 2, 4, fmt, out=b["P"], ws=b["ws"])
+            for i, u in enumerate(units):
+                u["prep"]()
                 evs[2 * i + 1].record()
-                sq.linear(b["P"], b["w"], out=b["Y"])
+                u["gemm"]()
                 evs[2 * i + 2].record()
     torch.cuda.synchronize()
 
@@ -307,14 +360,14 @@ def run_sharq(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms, prep_ms, lin_ms = [], [[] for _ in bufs], [[] for _ in bufs]
+    step_ms, prep_ms, lin_ms = [], [[] for _ in units], [[] for _ in units]
     with ClockSampler(local) as clk:
         for _ in range(args.steps):
             flush.zero_()                    # L2 flushed between timed steps
             g.replay()
             torch.cuda.synchronize()
             step_ms.append(evs[0].elapsed_time(evs[-1]))
-            for i in range(len(bufs)):
+            for i in range(len(units)):
                 prep_ms[i].append(evs[2 * i].elapsed_time(evs[2 * i + 1]))
                 lin_ms[i].append(evs[2 * i + 1].elapsed_time(evs[2 * i + 2]))
     torch.cuda.synchronize()
@@ -327,47 +380,59 @@ def run_sharq(args):
         dist.barrier()
     clocks = clk.summary()
 
-    fl_step = flops_of(linears, M)
+    fl_step = sum(2.0 * u["rows"] * u["N"] * u["K"] for u in units)
     ms_step = total_ms / args.steps
     value = fl_step * world * args.steps / (total_ms * 1e-3) / 1e12
-    tokens = M * world * args.steps / (total_ms * 1e-3)
+    tokens = tokens_per_step * world * args.steps / (total_ms * 1e-3)
 
     hbm, bf16, src = peaks()
     fp4_peak = 4.0 * bf16           # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PFLOP/s)
     lin_t = [statistics.mean(x) * 1e-3 for x in lin_ms]
     prep_t = [statistics.mean(x) * 1e-3 for x in prep_ms]
-    # Dominant kernel: the largest linear launch (gate+up).  Algorithmic
-    # dense-equivalent flops of the two-path linear at 2:4: 2MNK on the dense
-    # residual plus 2MNK*(n/m) on the sparse backbone at twice the rate.
-    dom = max(range(len(bufs)), key=lambda i: lin_t[i])
-    Ld = bufs[dom]["L"]
-    achieved = 2.5 * M * Ld.N * Ld.K / lin_t[dom] / 1e12
-    traffic = profiled_traffic(f"linear_{args.fmt}_{W.name}_{Ld.name}_M{M}",
-                               source_sha("linear.cu", "common.cuh"))
+    # Dominant kernel: the largest linear launch.  Algorithmic dense-equivalent
+    # flops of the two-path linear: 2MNK on the dense residual plus 2MNK*(n/m)
+    # on the n:m-sparse backbone at twice the dense rate.
+    alg_factor = 2.0 * (1.0 + 0.5 * n / m)
+    dom = max(range(len(units)), key=lambda i: lin_t[i])
+    ud = units[dom]
+    # roofline time = max(flops / FP4 peak, algorithmic bytes / HBM): weight codes
+    # + scales once, activation codes + scales of both paths, bf16 output
+    sfb = 1.0 / (16 if fmt == 0 else 32)
+    lin_bytes = (ud["N"] * ud["K"] * (0.5 + sfb) + ud["rows"] * ud["K"] * 2 * (0.5 + sfb)
+                 + 2.0 * ud["rows"] * ud["N"])
+    lin_flops = alg_factor * ud["rows"] * ud["N"] * ud["K"]
+    hbm_bound = lin_bytes / (hbm * 1e9) > lin_flops / (fp4_peak * 1e12)
+    if hbm_bound:
+        achieved, lin_peak, lin_unit = lin_bytes / lin_t[dom] / 1e9, hbm, "GB/s"
+    else:
+        achieved, lin_peak, lin_unit = lin_flops / lin_t[dom] / 1e12, fp4_peak, "TFLOP/s"
+    lin_key = f"linear_{args.fmt}_{args.workload}_{ud['name']}_M{args.M}"
+    traffic = profiled_traffic(lin_key, source_sha("linear.cu", "common.cuh"))
     # Prepare roofline on its largest launch (algorithmic bytes per element:
     # read X 2, backbone codes 0.5 (zero-filled) + scales, residual codes 0.5 + scales)
-    pdom = max(range(len(bufs)), key=lambda i: prep_t[i])
-    Lp = bufs[pdom]["L"]
-    prep_ach = PREP_BYTES_PER_ELEM[(fmt, 1)] * M * Lp.K / prep_t[pdom] / 1e9
-    prep_traffic = profiled_traffic(f"prepare_{args.fmt}_{W.name}_{Lp.name}_M{M}",
-                                    source_sha("prepare.cu", "common.cuh"))
+    bpe = PREP_BYTES_PER_ELEM[(fmt, 1)]
+    pdom = max(range(len(units)), key=lambda i: prep_t[i])
+    up_ = units[pdom]
+    prep_ach = bpe * up_["prep_rows"] * up_["K"] / prep_t[pdom] / 1e9
+    prep_key = f"prepare_{args.fmt}_{args.workload}_{up_['name']}_M{args.M}"
+    prep_traffic = profiled_traffic(prep_key, source_sha("prepare.cu", "common.cuh"))
 
     # end-to-end: host inputs (pinned) in, host outputs out, every step
     e2e = None
     if not args.no_e2e:
-        hx = [b["X"].cpu().pin_memory() for b in bufs]
-        hy = [torch.empty(b["Y"].shape, dtype=b["Y"].dtype, pin_memory=True) for b in bufs]
+        hx = [u["X"].cpu().pin_memory() for u in units]
+        hy = [torch.empty(u["Y"].shape, dtype=u["Y"].dtype, pin_memory=True) for u in units]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ts = []
         cur = torch.cuda.current_stream()
         for it in range(args.warmup + args.steps):
             flush.zero_()
             e0.record(cur)
-            for b, h in zip(bufs, hx):
-                b["X"].copy_(h, non_blocking=True)
+            for u, h in zip(units, hx):
+                u["X"].copy_(h, non_blocking=True)
             g.replay()
-            for b, h in zip(bufs, hy):
-                h.copy_(b["Y"], non_blocking=True)
+            for u, h in zip(units, hy):
+                h.copy_(u["Y"], non_blocking=True)
             e1.record(cur)
             torch.cuda.synchronize()
             if it >= args.warmup:
@@ -383,7 +448,8 @@ def run_sharq(args):
                "ms_per_step": tot / args.steps}
 
     base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "llama8b"):
+        linears = make_inputs(wl.WORKLOADS[args.workload], args.M)
         base = cpu_baseline(linears)
 
     if rank == 0:
@@ -392,29 +458,32 @@ def run_sharq(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4" if fmt == 0 else "mxfp4", "data": "synthetic",
-            "config": {"workload": f"{W.name}: Llama-3.1-8B-shaped decoder linears "
-                                   f"(qkv 4096x6144, o 4096x4096, gate_up 4096x28672, "
-                                   f"down 14336x4096), prefill M={M}, prepare+linear each",
-                       "M": M, "fmt": args.fmt, "nm": "2:4", "rmsnorm": "qkv, gate_up",
+            "config": {"workload": desc, "M": tokens_per_step, "fmt": args.fmt, "nm": args.nm,
                        "l2": "flushed between timed steps (512 MiB write)",
                        "timing": "CUDA graph per step, per-kernel external events"},
             "tokens_per_s": tokens,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic,
-                         "kernel": f"linear_kernel (two-path FP4 GEMM), {Ld.name} launch "
-                                   f"M={M} N={Ld.N} K={Ld.K}",
-                         "peak_note": f"dense FP4 = 4 x {src} bf16 burst ({bf16:.0f} TFLOP/s)",
-                         "achieved_note": "2.5*M*N*K per launch (2:4 backbone at 2x rate + dense residual)"},
+            "roofline": {"bound": "hbm" if hbm_bound else "tensor", "achieved": achieved,
+                         "peak": lin_peak, "unit": lin_unit, "frac": achieved / lin_peak,
+                         "traffic": traffic, "algorithmic_bytes": lin_bytes,
+                         "algorithmic_flops": lin_flops,
+                         "kernel": f"{'moe_' if wl.WORKLOADS[args.workload].moe else ''}linear_kernel "
+                                   f"(two-path FP4 GEMM), {ud['name']} launch rows={ud['rows']} "
+                                   f"N={ud['N']} K={ud['K']}",
+                         "peak_note": (f"{src} copy bandwidth" if hbm_bound else
+                                       f"dense FP4 = 4 x {src} bf16 burst ({bf16:.0f} TFLOP/s)"),
+                         "achieved_note": f"{alg_factor:g}*M*N*K per launch ({n}:{m} backbone at 2x "
+                                          f"rate + dense residual)"},
             "prepare_roofline": {"bound": "hbm", "achieved": prep_ach, "peak": hbm, "unit": "GB/s",
                                  "frac": prep_ach / hbm, "traffic": prep_traffic,
-                                 "kernel": f"prepare_kernel, {Lp.name} launch M={M} K={Lp.K}",
-                                 "bytes_per_elem": PREP_BYTES_PER_ELEM[(fmt, 1)],
-                                 "peak_note": f"{src} copy bandwidth"},
-            "kernel_ms": {b["L"].name: {"prepare": statistics.mean(p), "linear": statistics.mean(l)}
-                          for b, p, l in zip(bufs, prep_ms, lin_ms)},
-            "executed_fp4_tflops": sum(4.0 * M * b["L"].N * b["L"].K for b in bufs) / sum(lin_t) / 1e12,
-            "prepare_gbs_all": sum(PREP_BYTES_PER_ELEM[(fmt, 1)] * M * b["L"].K for b in bufs) / sum(prep_t) / 1e9,
-            "gpu_launches": 2 * len(bufs) * args.steps,
+                                 "kernel": f"prepare_kernel, {up_['name']} launch rows={up_['prep_rows']} "
+                                           f"K={up_['K']}",
+                                 "bytes_per_elem": bpe, "peak_note": f"{src} copy bandwidth"},
+            "kernel_ms": {u["name"]: {"prepare": statistics.mean(p), "linear": statistics.mean(l)}
+                          for u, p, l in zip(units, prep_ms, lin_ms)},
+            "executed_fp4_tflops": sum(4.0 * u["rows"] * u["N"] * u["K"] for u in units) / sum(lin_t) / 1e12,
+            "prepare_gbs_all": sum(bpe * u["prep_rows"] * u["K"] for u in units) / sum(prep_t) / 1e9,
+            "gpu_launches": (2 * len(units) + (len(units) if wl.WORKLOADS[args.workload].moe else 0))
+                            * args.steps,
             "device_status": status,
             "clocks": clocks,
             "e2e": e2e,
@@ -430,6 +499,9 @@ def run_sharq(args):
 
 def main():
     args = parse_args()
+    if args.M is None:
+        Ms = wl.WORKLOADS[args.workload].Ms
+        args.M = 2048 if args.workload == "llama8b" else (Ms[0] if Ms else 0)
     if args.impl == "reference":
         return run_reference(args)
     return run_sharq(args)
