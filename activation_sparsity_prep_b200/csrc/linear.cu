@@ -28,7 +28,7 @@ namespace {
 
 constexpr int BM = 128, BN = 128, BK = 256;   // BK in FP4 elements = 128 bytes per row
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTileBytes = BM * (BK / 2);  // 16 KiB per operand tile
 constexpr uint32_t kTmemCols = 512;
 
@@ -48,7 +48,8 @@ struct Cfg {
 
 struct alignas(8) Barriers {
     uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t empty[kStages];      // MMAs done (tcgen05.commit) + scale warps done reading
+    uint64_t sf_full[kStages];    // scale factors of the stage are in tensor memory
     uint64_t acc_full;      // MMAs of the current tile done (tcgen05.commit)
     uint64_t acc_empty;     // epilogue has drained the accumulators (4 warps)
     uint32_t tmem_base;
@@ -208,7 +209,11 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     sched_prepare(sc, ssm);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1 + 4);
+            mbar_init(&bars->sf_full[s], 4);
+        }
         mbar_init(&bars->acc_full, 1);
         mbar_init(&bars->acc_empty, 4);
         fence_barrier_init();
@@ -220,9 +225,14 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     const int ntiles = sched_count(sc, ssm);
     const uint32_t tmem = bars->tmem_base;
     const uint32_t t_acc_b = tmem, t_acc_r = tmem + BN;
-    const uint32_t t_sfa_b = tmem + 2 * BN;
-    const uint32_t t_sfa_r = t_sfa_b + 4 * C::kAtoms;
-    const uint32_t t_sfb = t_sfa_r + 4 * C::kAtoms;
+    // Scale factors: one tensor-memory buffer per pipeline stage, written by
+    // the four scale warps (warps 6..9) with tcgen05.st, each into its own
+    // 32-lane quarter -- which also gives the replication across quarters
+    // that the block-scaled MMA reads.  Copying them with tcgen05.cp would
+    // put 3 * kAtoms copies per stage into the MMA issue stream, where they
+    // do not overlap the MMAs.
+    constexpr uint32_t kSfColsPerStage = 3 * 4 * C::kAtoms;
+    static_assert(2 * BN + kStages * kSfColsPerStage <= kTmemCols, "tensor memory budget");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -260,18 +270,14 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars->sf_full[s], (it / kStages) & 1)) { ok = false; break; }
                     tc_fence_after();
                     uint8_t* st = smem + s * C::kStageStride;
                     const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + kTileBytes);
                     const uint32_t a_w = smem_u32(st + 2 * kTileBytes);
-                    const uint32_t s_b = smem_u32(st + 3 * kTileBytes);
-                    const uint32_t s_r = s_b + C::kSfBytes, s_w = s_b + 2 * C::kSfBytes;
-#pragma unroll
-                    for (int at = 0; at < C::kAtoms; ++at) {
-                        tc_cp_32x128b_warpx4(t_sfa_b + 4 * at, sdesc_sf_atom(s_b + 512 * at));
-                        tc_cp_32x128b_warpx4(t_sfa_r + 4 * at, sdesc_sf_atom(s_r + 512 * at));
-                        tc_cp_32x128b_warpx4(t_sfb + 4 * at, sdesc_sf_atom(s_w + 512 * at));
-                    }
+                    const uint32_t t_sfa_b = tmem + 2 * BN + s * kSfColsPerStage;
+                    const uint32_t t_sfa_r = t_sfa_b + 4 * C::kAtoms;
+                    const uint32_t t_sfb = t_sfa_r + 4 * C::kAtoms;
 #pragma unroll
                     for (int j = 0; j < BK / 64; ++j) {
                         const int at = j / C::kStepsPerAtom;
@@ -287,6 +293,30 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                     tc_commit(&bars->empty[s]);
                 }
                 tc_commit(&bars->acc_full);
+            }
+        }
+    } else if (warp >= 6) {
+        // Scale warps: warp w writes lane quarter w%4; lane l copies row l of
+        // every 32-row x 16-byte scale atom of the stage into 4 columns.
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const uint32_t s = it % kStages;
+                if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
+                const uint8_t* sf = smem + s * C::kStageStride + 3 * kTileBytes;
+                const uint32_t tcol = tmem + 2 * BN + s * kSfColsPerStage + lane_off;
+#pragma unroll
+                for (int o = 0; o < 3; ++o)
+#pragma unroll
+                    for (int at = 0; at < C::kAtoms; ++at)
+                        tmem_st_32x32b_x4(tcol + o * 4 * C::kAtoms + 4 * at,
+                                          ld_shared_v4(sf + o * C::kSfBytes + 512 * at + 16 * lane));
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) { mbar_arrive(&bars->sf_full[s]); mbar_arrive(&bars->empty[s]); }
             }
         }
     } else {
