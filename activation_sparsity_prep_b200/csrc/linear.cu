@@ -108,10 +108,17 @@ struct Sched {
     int N;
 };
 
-struct SchedSmem {
+struct SchedTables {
     int off[kMaxExperts + 1];    // dispatch offsets
     int poff[kMaxExperts + 1];   // padded row offsets (128-aligned)
     int tpre[kMaxExperts + 1];   // tile prefix
+};
+
+// The grouped form uses the scheduler tables; the plain form uses the same
+// bytes as four 2 KiB epilogue staging buffers (one per epilogue warp).
+union SchedSmem {
+    SchedTables t;
+    uint8_t stage[4][2048];
 };
 
 __device__ __forceinline__ int ceil128(int x) { return (x + 127) >> 7; }
@@ -127,7 +134,7 @@ __device__ void sched_prepare(const Sched& sc, SchedSmem* sm) {
             int cnt = 0;
             if (e < sc.E) {
                 const int o0 = sc.offsets[e], o1 = sc.offsets[e + 1];
-                sm->off[e] = o0;
+                sm->t.off[e] = o0;
                 cnt = o1 - o0;
             }
             int pr = ceil128(cnt) * 128, tl = ceil128(cnt) * sc.nt_count;
@@ -137,20 +144,20 @@ __device__ void sched_prepare(const Sched& sc, SchedSmem* sm) {
                 int vp = __shfl_up_sync(0xffffffffu, ip, o), vt = __shfl_up_sync(0xffffffffu, it, o);
                 if (lane >= o) { ip += vp; it += vt; }
             }
-            if (e < sc.E) { sm->poff[e] = carry_p + ip - pr; sm->tpre[e] = carry_t + it - tl; }
+            if (e < sc.E) { sm->t.poff[e] = carry_p + ip - pr; sm->t.tpre[e] = carry_t + it - tl; }
             carry_p += __shfl_sync(0xffffffffu, ip, 31);
             carry_t += __shfl_sync(0xffffffffu, it, 31);
         }
         if (lane == 0) {
-            sm->off[sc.E] = sc.offsets[sc.E];
-            sm->poff[sc.E] = carry_p;
-            sm->tpre[sc.E] = carry_t;
+            sm->t.off[sc.E] = sc.offsets[sc.E];
+            sm->t.poff[sc.E] = carry_p;
+            sm->t.tpre[sc.E] = carry_t;
         }
     }
 }
 
 __device__ __forceinline__ int sched_count(const Sched& sc, const SchedSmem* sm) {
-    return sc.grouped ? sm->tpre[sc.E] : sc.mt_count * sc.nt_count;
+    return sc.grouped ? sm->t.tpre[sc.E] : sc.mt_count * sc.nt_count;
 }
 
 __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem* sm, int t) {
@@ -169,17 +176,17 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
     int lo = 0, hi = sc.E;                          // largest e with tpre[e] <= t
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (sm->tpre[mid] <= t) lo = mid; else hi = mid;
+        if (sm->t.tpre[mid] <= t) lo = mid; else hi = mid;
     }
     const int e = lo;
-    const int cnt = sm->off[e + 1] - sm->off[e];
+    const int cnt = sm->t.off[e + 1] - sm->t.off[e];
     const int mtn = ceil128(cnt);
-    const int local = t - sm->tpre[e];
+    const int local = t - sm->t.tpre[e];
     const int nt = local / mtn, mt = local - nt * mtn;
-    ti.a_row = sm->poff[e] + (int64_t)mt * 128;
+    ti.a_row = sm->t.poff[e] + (int64_t)mt * 128;
     ti.w_row = (int64_t)e * sc.N + (int64_t)nt * 128;
     ti.w_sf = (int64_t)e * sc.w_sf_stride + (int64_t)nt * (sc.nsf / 4) * 512;
-    ti.y_row = sm->off[e] + (int64_t)mt * 128;
+    ti.y_row = sm->t.off[e] + (int64_t)mt * 128;
     ti.rows = min(128, cnt - mt * 128);
     ti.col = nt * 128;
     ti.e = e;
@@ -201,7 +208,9 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Barriers* bars = reinterpret_cast<Barriers*>(smem + kStages * C::kStageStride);
-    SchedSmem* ssm = reinterpret_cast<SchedSmem*>(reinterpret_cast<uint8_t*>(bars) + sizeof(Barriers));
+    // 128-byte aligned: the staging buffers take 16-byte vector stores
+    SchedSmem* ssm = reinterpret_cast<SchedSmem*>(
+        (reinterpret_cast<uintptr_t>(bars) + sizeof(Barriers) + 127) & ~uintptr_t(127));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = K / BK;
@@ -380,12 +389,39 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->acc_empty);
-                if (row_ok) {
-                    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(ep.Y) + row * ep.N + col0;
+                if (sc.grouped) {
+                    // rows past the group belong to the next expert: masked row stores
+                    if (row_ok) {
+                        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(ep.Y) + row * ep.N + col0;
 #pragma unroll
-                    for (int i = 0; i < BN / 8; ++i)
-                        *reinterpret_cast<uint4*>(y + 8 * i) =
-                            make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+                        for (int i = 0; i < BN / 8; ++i)
+                            *reinterpret_cast<uint4*>(y + 8 * i) =
+                                make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+                    }
+                } else {
+                    // Stage each 32-row x 32-column chunk in shared memory so
+                    // that every store instruction writes 8 rows x 64
+                    // contiguous bytes instead of 32 rows x 16 bytes.
+                    uint8_t* stg = ssm->stage[q];
+                    const int64_t wrow0 = ti.y_row + q * 32;
+#pragma unroll
+                    for (int cc = 0; cc < BN / 32; ++cc) {
+#pragma unroll
+                        for (int p = 0; p < 4; ++p)
+                            *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (p ^ (lane & 3))) =
+                                make_uint4(out[cc * 16 + 4 * p], out[cc * 16 + 4 * p + 1],
+                                           out[cc * 16 + 4 * p + 2], out[cc * 16 + 4 * p + 3]);
+                        __syncwarp();
+#pragma unroll
+                        for (int st8 = 0; st8 < 4; ++st8) {
+                            const int r = 8 * st8 + (lane >> 2), p = lane & 3;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (p ^ (r & 3)));
+                            if (q * 32 + r < ti.rows)
+                                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(ep.Y) +
+                                                          (wrow0 + r) * ep.N + col0 + cc * 32 + p * 8) = v;
+                        }
+                        __syncwarp();
+                    }
                 }
             }
         }
@@ -430,7 +466,7 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_b
 
 template <int FMT>
 size_t linear_smem_bytes() {
-    return kStages * Cfg<FMT>::kStageStride + sizeof(Barriers) + sizeof(SchedSmem) + 1024;
+    return kStages * Cfg<FMT>::kStageStride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
 }
 
 template <int FMT>
@@ -504,10 +540,10 @@ moe_gather_kernel(const uint8_t* __restrict__ bb_codes, const uint8_t* __restric
         int lo = 0, hi = sc.E;                      // expert of row t
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (ssm.off[mid] <= t) lo = mid; else hi = mid;
+            if (ssm.t.off[mid] <= t) lo = mid; else hi = mid;
         }
         const int64_t src = row_index ? (int64_t)row_index[t] : t;
-        const int64_t dst = ssm.poff[lo] + (t - ssm.off[lo]);
+        const int64_t dst = ssm.t.poff[lo] + (t - ssm.t.off[lo]);
         const uint4* sb = reinterpret_cast<const uint4*>(bb_codes + src * row_bytes);
         const uint4* sr = reinterpret_cast<const uint4*>(rs_codes + src * row_bytes);
         uint4* db = reinterpret_cast<uint4*>(gb_codes + dst * row_bytes);
