@@ -134,14 +134,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the hardware may suspend the thread until the phase
+// completes or about hint_ns nanoseconds pass, instead of returning at once:
+// a waiting warp then takes no issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false (and records a timeout)
 // when the phase does not complete within about a second.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long t0 = globaltimer();
     while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
         if (globaltimer() - t0 > kWaitLimitNs) {
             record_status(kStatusMbarTimeout);
             return false;

@@ -61,6 +61,10 @@ CASES = [
     (129, 1024, "laplace_outlier", "ones", 1, 4, "mxfp4"),
     (33, 768, "student_t", None, 4, 8, "mxfp4"),
     (200, 4096, "laplace_outlier", "random", 2, 4, "mxfp4"),
+    # several hundred rows: many CTAs per phase, ragged last CTA
+    (1024, 4096, "laplace_outlier", "ones", 2, 4, "mxfp4"),
+    (600, 4096, "student_t", None, 1, 4, "nvfp4"),
+    (700, 3584, "student_t", "random", 4, 8, "nvfp4"),
 ]
 
 
