@@ -70,7 +70,10 @@ def lib() -> ctypes.CDLL:
             L.orc_mask.argtypes = [P, i64, i32, i32, i32, P]
             L.orc_quant_nvfp4.argtypes = [P, i64, i32, P, P, P, P]
             L.orc_quant_mxfp4.argtypes = [P, i64, i32, P, P, P, P]
-            L.orc_prepare.argtypes = [P, P, f32, i64, i32, i32, i32, i32,
+            L.orc_quant_nvfp4_amax.argtypes = [P, i64, i32, f32, P, P, P, P]
+            L.orc_tensor_amax.argtypes = [P, i64]
+            L.orc_tensor_amax.restype = f32
+            L.orc_prepare.argtypes = [P, P, f32, i64, i32, i32, i32, i32, i32,
                                       P, P, P, P, P, P, P, P, P]
             L.orc_prepare.restype = i32
             L.orc_quantize_weight.argtypes = [P, i64, i32, i32, P, P, P]
@@ -184,10 +187,17 @@ class Prepared:
     r: Optional[np.ndarray] = None
 
 
+RESIDUAL_SCALES = {"own": 0, "shared": 1}
+
+
 def prepare(X: np.ndarray, gamma: Optional[np.ndarray], eps: float = 1e-6,
-            n: int = 2, m: int = 4, fmt="nvfp4", keep_intermediates: bool = False
-            ) -> Prepared:
-    """The preparation operator on a whole tensor X [M, K] (bf16 bits)."""
+            n: int = 2, m: int = 4, fmt="nvfp4", keep_intermediates: bool = False,
+            residual_scale: str = "own") -> Prepared:
+    """The preparation operator on a whole tensor X [M, K] (bf16 bits).
+
+    residual_scale "own": the residual is quantised with its own tensor
+    scale (the plain reading of the abstract); "shared": with the backbone's
+    (NVFP4 only; MXFP4 has no tensor scale, so both settings agree)."""
     fmt = _fmt(fmt)
     X = np.ascontiguousarray(X, dtype=np.uint16)
     M, K = X.shape
@@ -202,7 +212,8 @@ def prepare(X: np.ndarray, gamma: Optional[np.ndarray], eps: float = 1e-6,
     rg = np.zeros(1, dtype=np.float32)
     y = np.empty((M, K), dtype=np.float32) if keep_intermediates else None
     r = np.empty((M, K), dtype=np.float32) if keep_intermediates else None
-    rc_ = lib().orc_prepare(_p(X), _p(g), eps, M, K, n, m, fmt, _p(mk),
+    rc_ = lib().orc_prepare(_p(X), _p(g), eps, M, K, n, m, fmt,
+                            RESIDUAL_SCALES[residual_scale], _p(mk),
                             _p(bc), _p(bs), _p(bg), _p(rc), _p(rsc), _p(rg),
                             _p(y), _p(r))
     if rc_ != 0:

@@ -229,13 +229,27 @@ void orc_mask(const float* y, int64_t M, int K, int n, int m, uint8_t* keep) {
 /* NVFP4: A = max|T|; G_enc = 2688/A, G_dec = A/2688 (both 1 when A = 0),
  * 2688 = 6 * 448; K1 = G_enc/6; per 16-block e = E4M3(b*K1);
  * inv = G_enc/e (0 when e = 0); q = E2M1(T*inv); D = (val(q)*e)*G_dec. */
-void orc_quant_nvfp4(const float* T, int64_t R, int K,
-                     uint8_t* codes, uint8_t* scales, float* gdec_out, float* D) {
+float orc_tensor_amax(const float* T, int64_t n) {
     float A = 0.0f;
-    for (int64_t i = 0; i < R * (int64_t)K; ++i) {
+    for (int64_t i = 0; i < n; ++i) {
         float a = fabsf(T[i]);
         if (a > A) A = a;
     }
+    return A;
+}
+
+/* The same quantiser with the tensor amax A given by the caller instead of
+ * taken over T (the shared-scale residual below uses the backbone's A). */
+void orc_quant_nvfp4_amax(const float* T, int64_t R, int K, float A,
+                          uint8_t* codes, uint8_t* scales, float* gdec_out, float* D);
+
+void orc_quant_nvfp4(const float* T, int64_t R, int K,
+                     uint8_t* codes, uint8_t* scales, float* gdec_out, float* D) {
+    orc_quant_nvfp4_amax(T, R, K, orc_tensor_amax(T, R * (int64_t)K), codes, scales, gdec_out, D);
+}
+
+void orc_quant_nvfp4_amax(const float* T, int64_t R, int K, float A,
+                          uint8_t* codes, uint8_t* scales, float* gdec_out, float* D) {
     float genc = 1.0f, gdec = 1.0f;
     if (A != 0.0f) { genc = 2688.0f / A; gdec = A / 2688.0f; }
     float k1 = genc / 6.0f;
@@ -309,14 +323,17 @@ static void quant(int fmt, const float* T, int64_t R, int K,
 /* against the dequantised backbone + residual FP4, one operator):           */
 /*   y = norm(x); keep = mask(y); B = keep ? y : +0;                         */
 /*   (codes_b, scales_b, G_b, D_b) = Q(B); r = y - D_b;                      */
-/*   (codes_r, scales_r, G_r) = Q(r)   -- residual has its own tensor scale. */
+/*   (codes_r, scales_r, G_r) = Q(r)   -- residual has its own tensor scale, */
+/*   or, with residual_shared (NVFP4), the backbone's: Q(r) is taken with    */
+/*   A = max|B| in place of max|r|, so G_r = G_b (a variant the pages leave  */
+/*   open: the abstract names one tensor scale per FP4 tensor or none).      */
 /* mask_bits [M, K/8] (bit t of byte j = element 8j+t kept) is optional, as  */
 /* are the y / r outputs used by invariant tests.                            */
 /* Returns 0, or -1 on a bad argument or allocation failure.                 */
 /* ------------------------------------------------------------------------ */
 
 int orc_prepare(const uint16_t* X, const uint16_t* gamma, float eps,
-                int64_t M, int K, int n, int m, int fmt,
+                int64_t M, int K, int n, int m, int fmt, int residual_shared,
                 uint8_t* mask_bits,
                 uint8_t* bb_codes, uint8_t* bb_scales, float* bb_g,
                 uint8_t* rs_codes, uint8_t* rs_scales, float* rs_g,
@@ -332,10 +349,12 @@ int orc_prepare(const uint16_t* X, const uint16_t* gamma, float eps,
     orc_normalize(X, gamma, eps, M, K, y);
     orc_mask(y, M, K, n, m, keep);
     for (int64_t i = 0; i < E; ++i) B[i] = keep[i] ? y[i] : 0.0f;
+    const float A_b = orc_tensor_amax(B, E);
     quant(fmt, B, M, K, bb_codes, bb_scales, bb_g, D);
     float* r = B;                                /* reuse: B is no longer needed */
     for (int64_t i = 0; i < E; ++i) r[i] = y[i] - D[i];
-    quant(fmt, r, M, K, rs_codes, rs_scales, rs_g, NULL);
+    if (residual_shared && fmt == ORC_NVFP4) orc_quant_nvfp4_amax(r, M, K, A_b, rs_codes, rs_scales, rs_g, NULL);
+    else                                     quant(fmt, r, M, K, rs_codes, rs_scales, rs_g, NULL);
     if (r_out) memcpy(r_out, r, sizeof(float) * (size_t)E);
     if (mask_bits) {
         for (int64_t i = 0; i < M; ++i)

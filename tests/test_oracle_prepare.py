@@ -294,3 +294,74 @@ def test_moe_reduces_to_per_expert_linear():
         e = int(np.searchsorted(off, t, side="right") - 1)
         want = oracle.linear(oracle.gather_rows(P, ri[t:t + 1]), experts[e])[0]
         assert np.array_equal(Y[t], want)
+
+
+# ---------------------------------------------------------------------------
+# Residual quantised with the backbone's tensor scale ("shared" variant).
+# ---------------------------------------------------------------------------
+
+def _row32(vals):
+    x = np.zeros((1, 32), dtype=np.float32)
+    for k, v in vals.items():
+        x[0, k] = v
+    return wl.f32_to_bf16_bits(x)
+
+
+def test_shared_residual_scale_worked_example():
+    """One row, K = 32, no norm, 2:4, NVFP4; worked by hand.
+
+    Backbone: element 0 = 2688 (with element 1 = 0 kept beside it; every
+    all-zero group keeps its first two slots), and the
+    group [768, 384, 384, 0] at elements 16..19 keeps 768 and the first 384.
+    A_b = 2688, so G_enc = 1, G_dec = 1, K1 = fl(1/6); block 0 gets
+    E4M3(fl(2688 K1)) = 448 (0x7E) and block 1 E4M3(fl(768 K1) = 128) = 0x70;
+    every kept value is exactly on its grid, so the residual is zero except
+    r[18] = 384 (the pruned 384).
+    Own residual scale: A_r = 384, G_enc = 7, K1 = fl(7/6) and
+    fl(384 fl(7/6)) is 448 - 2^-16, a tie that rounds to even 448: block
+    scale 0x7E, G_r = fl(384/2688) = fl(1/7).
+    Shared: A = A_b = 2688, fl(384 fl(1/6)) = 64: block scale 0x68 (64),
+    G_r = 1.  Either way r[18] / scale-product is exactly 6 -> code 7."""
+    X = _row32({0: 2688.0, 16: 768.0, 17: 384.0, 18: 384.0})
+    own = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4", residual_scale="own")
+    sh = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4", residual_scale="shared")
+    for P in (own, sh):
+        # every group keeps its first two slots here (all-zero groups too)
+        assert list(P.mask[0]) == [0x33] * 4
+        assert list(P.bb.scales[0]) == [0x7E, 0x70]
+        assert float(P.bb.tscale) == 1.0
+        rc = P.rs.codes[0]
+        assert rc[9] == 0x07 and np.count_nonzero(rc) == 1             # element 18: code 7 (6.0)
+        assert P.rs.scales[0, 0] == 0
+    assert own.rs.scales[0, 1] == 0x7E
+    assert np.float32(own.rs.tscale) == np.float32(384.0) / np.float32(2688.0)
+    assert sh.rs.scales[0, 1] == 0x68
+    assert float(sh.rs.tscale) == 1.0
+
+
+def test_shared_equals_own_when_a_pruned_entry_ties_the_max():
+    """If a pruned element's |y| equals the tensor maximum, max|r| = max|B|,
+    so the two settings must give the same residual bit for bit."""
+    X = wl.activation("laplace_outlier", 61, 0, 8, 256).copy()
+    big = wl.f32_to_bf16_bits(np.array([[3000.0]], dtype=np.float32))[0, 0]
+    X[3, 40:43] = big            # group 40..43: two of the three equal maxima are kept
+    X[3, 43] = 0
+    own = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4", residual_scale="own")
+    sh = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4", residual_scale="shared")
+    assert np.array_equal(own.rs.codes, sh.rs.codes)
+    assert np.array_equal(own.rs.scales, sh.rs.scales)
+    assert np.float32(own.rs.tscale) == np.float32(sh.rs.tscale)
+
+
+def test_shared_residual_tensor_scale_is_the_backbones():
+    X = wl.activation("laplace_outlier", 62, 0, 33, 512)
+    for g in (None, wl.gamma_ones(512)):
+        sh = oracle.prepare(X, g, 1e-6, 2, 4, "nvfp4", residual_scale="shared")
+        own = oracle.prepare(X, g, 1e-6, 2, 4, "nvfp4", residual_scale="own")
+        assert np.float32(sh.rs.tscale).view(np.uint32) == np.float32(sh.bb.tscale).view(np.uint32)
+        assert np.array_equal(sh.bb.codes, own.bb.codes) and np.array_equal(sh.mask, own.mask)
+        assert not np.array_equal(sh.rs.scales, own.rs.scales)     # a real difference on real data
+    # MXFP4 has no tensor scale: the setting changes nothing
+    a = oracle.prepare(X, None, 1e-6, 2, 4, "mxfp4", residual_scale="own")
+    b = oracle.prepare(X, None, 1e-6, 2, 4, "mxfp4", residual_scale="shared")
+    assert np.array_equal(a.rs.codes, b.rs.codes) and np.array_equal(a.rs.scales, b.rs.scales)
