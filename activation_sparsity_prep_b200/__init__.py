@@ -50,7 +50,8 @@ class _Prepared(ctypes.Structure):
                 ("bb_tscale", ctypes.c_void_p), ("rs_codes", ctypes.c_void_p),
                 ("rs_scales", ctypes.c_void_p), ("rs_tscale", ctypes.c_void_p),
                 ("mask", ctypes.c_void_p), ("M", ctypes.c_int), ("K", ctypes.c_int),
-                ("n", ctypes.c_int), ("m", ctypes.c_int), ("fmt", ctypes.c_int)]
+                ("n", ctypes.c_int), ("m", ctypes.c_int), ("fmt", ctypes.c_int),
+                ("residual_scale", ctypes.c_int)]
 
 
 _lib = None
@@ -101,6 +102,13 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
 
 def _fmt(fmt) -> int:
     return _FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+_RESIDUAL = {"own": 0, "shared": 1}
+
+
+def _residual(rs) -> int:
+    return _RESIDUAL[rs] if isinstance(rs, str) else int(rs)
 
 
 def _ptr(t) -> Optional[int]:
@@ -167,15 +175,17 @@ class Prepared:
     n: int
     m: int
     fmt: int
+    residual_scale: int = 0      # 0 own, 1 shared with the backbone (NVFP4)
 
     def _c(self) -> _Prepared:
         return _Prepared(_ptr(self.bb_codes), _ptr(self.bb_scales), _ptr(self.bb_tscale),
                          _ptr(self.rs_codes), _ptr(self.rs_scales), _ptr(self.rs_tscale),
-                         _ptr(self.mask), self.M, self.K, self.n, self.m, self.fmt)
+                         _ptr(self.mask), self.M, self.K, self.n, self.m, self.fmt,
+                         self.residual_scale)
 
     @staticmethod
     def empty(M: int, K: int, n: int = 2, m: int = 4, fmt="nvfp4", want_mask: bool = False,
-              device="cuda") -> "Prepared":
+              device="cuda", residual_scale="own") -> "Prepared":
         import torch
         f = _fmt(fmt)
         sb = scale_bytes(M, K, f)
@@ -185,7 +195,7 @@ class Prepared:
                         torch.empty((M, K // 2), **u8), torch.empty((sb,), **u8),
                         torch.empty((1,), dtype=torch.float32, device=device),
                         torch.empty((M, K // 8), **u8) if want_mask else None,
-                        M, K, n, m, f)
+                        M, K, n, m, f, _residual(residual_scale))
 
 
 def _workspace(M: int, K: int, fmt: int, ws=None, device="cuda"):
@@ -212,12 +222,15 @@ def quantize_weight(W, fmt="nvfp4", out: Optional[Weight] = None, ws=None, strea
 
 def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4",
             want_mask: bool = False, out: Optional[Prepared] = None, ws=None,
-            stream=None) -> Prepared:
-    """X: bf16 [M, K] device tensor; gamma: bf16 [K] or None (no norm)."""
+            stream=None, residual_scale="own") -> Prepared:
+    """X: bf16 [M, K] device tensor; gamma: bf16 [K] or None (no norm).
+    residual_scale: "own" or "shared" (ignored when ``out`` is given: the
+    output's own setting applies)."""
     L = load_sharq_ops()
     M, K = X.shape
     f = _fmt(fmt)
-    p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device)
+    p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
+                                                   residual_scale=residual_scale)
     ws = _workspace(M, K, f, ws, X.device)
     cp = p._c()
     _check("sharq_prepare",

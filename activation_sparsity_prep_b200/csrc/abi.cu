@@ -92,6 +92,8 @@ sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps
     const sharq_prepared& o = *out;
     if (!valid_fmt(o.fmt) || !valid_shape(o.M, o.K)) return SHARQ_ERR_INVALID_ARG;
     if (!(o.m == 2 || o.m == 4 || o.m == 8) || o.n < 1 || o.n > o.m) return SHARQ_ERR_INVALID_ARG;
+    if (o.residual_scale != SHARQ_RESIDUAL_OWN && o.residual_scale != SHARQ_RESIDUAL_SHARED)
+        return SHARQ_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !(eps < 1e30f)) return SHARQ_ERR_INVALID_ARG;
     if (!o.bb_tscale || !o.rs_tscale) return SHARQ_ERR_INVALID_ARG;
     if (o.M > 0 && (!X_bf16 || !o.bb_codes || !o.bb_scales || !o.rs_codes || !o.rs_scales))
@@ -104,7 +106,7 @@ sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps
     if (ws_bytes < sharq::prepare_ws_bytes(o.M)) return SHARQ_ERR_INVALID_ARG;
     sharq::PrepareLaunch p{};
     p.X = X_bf16; p.gamma = gamma_bf16; p.eps = eps; p.M = o.M; p.K = o.K; p.n = o.n; p.m = o.m;
-    p.fmt = o.fmt; p.weight = false;
+    p.fmt = o.fmt; p.weight = false; p.residual_shared = o.residual_scale == SHARQ_RESIDUAL_SHARED;
     p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
     p.rs_codes = o.rs_codes; p.rs_scales = o.rs_scales; p.rs_tscale = o.rs_tscale;
     p.mask = o.mask; p.ws = ws;
@@ -115,6 +117,8 @@ sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps
 static sharq_status check_linear_args(const sharq_prepared* x, const sharq_weight* w, void* Y) {
     if (!x || !w || (!Y && x->M > 0)) return SHARQ_ERR_INVALID_ARG;
     if (!valid_fmt(x->fmt) || x->fmt != w->fmt) return SHARQ_ERR_INVALID_ARG;
+    if (x->residual_scale != SHARQ_RESIDUAL_OWN && x->residual_scale != SHARQ_RESIDUAL_SHARED)
+        return SHARQ_ERR_INVALID_ARG;
     if (!valid_shape(x->M, x->K) || x->K != w->K) return SHARQ_ERR_INVALID_ARG;
     if (w->N <= 0 || w->N % 128 != 0) return SHARQ_ERR_INVALID_ARG;
     if (!x->bb_tscale || !x->rs_tscale || !w->codes || !w->scales || !w->tensor_scale)
@@ -137,6 +141,7 @@ sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w, void* 
     p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
     p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
     p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
+    p.one_acc = x->fmt == SHARQ_MXFP4 || x->residual_scale == SHARQ_RESIDUAL_SHARED;
     return cuda_status(sharq::launch_linear(p, static_cast<cudaStream_t>(stream),
                                             sharq::device_sm_count()));
 }
@@ -156,6 +161,8 @@ sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
     if (T > 0 && (!Y || !ws)) return SHARQ_ERR_INVALID_ARG;
     if (!valid_fmt(x->fmt) || x->fmt != w->fmt || !valid_shape(x->M, x->K) || x->K != w->K)
         return SHARQ_ERR_INVALID_ARG;
+    if (x->residual_scale != SHARQ_RESIDUAL_OWN && x->residual_scale != SHARQ_RESIDUAL_SHARED)
+        return SHARQ_ERR_INVALID_ARG;
     if (w->N <= 0 || w->N % 128 != 0 || !w->codes || !w->scales || !w->tensor_scale)
         return SHARQ_ERR_INVALID_ARG;
     if (!x->bb_tscale || !x->rs_tscale) return SHARQ_ERR_INVALID_ARG;
@@ -172,6 +179,7 @@ sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
     p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
     p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
     p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
+    p.one_acc = x->fmt == SHARQ_MXFP4 || x->residual_scale == SHARQ_RESIDUAL_SHARED;
     p.row_index = row_index; p.offsets = expert_offsets; p.E = E; p.T = T; p.ws = ws;
     return cuda_status(sharq::launch_moe_linear(p, static_cast<cudaStream_t>(stream),
                                                 sharq::device_sm_count()));

@@ -262,6 +262,21 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
                  :: "r"(taddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
+// 8 or 16 consecutive columns per lane in one store (two or four uint4).
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint4 (&v)[2]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "r"(taddr), "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w),
+                    "r"(v[1].x), "r"(v[1].y), "r"(v[1].z), "r"(v[1].w) : "memory");
+}
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint4 (&v)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, "
+                 "%9, %10, %11, %12, %13, %14, %15, %16};"
+                 :: "r"(taddr), "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w),
+                    "r"(v[1].x), "r"(v[1].y), "r"(v[1].z), "r"(v[1].w),
+                    "r"(v[2].x), "r"(v[2].y), "r"(v[2].z), "r"(v[2].w),
+                    "r"(v[3].x), "r"(v[3].y), "r"(v[3].z), "r"(v[3].w) : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -9,12 +9,17 @@
 //   acc_b += A_b x W^T,   acc_r += A_r x W^T.
 // The epilogue reads both accumulators back and writes
 //   Y = G_w * (G_b * acc_b + G_r * acc_r)
-// as bf16 (or fp32).  The backbone runs as a dense MMA over zero-filled codes:
+// as bf16 (or fp32).  When the two tensor scales are equal by construction
+// (MXFP4, or a residual quantised against the backbone's tensor scale) both
+// MMAs accumulate into one accumulator, Y = G_w * G_b * acc, and the two
+// tensor-memory accumulators serve as a double buffer instead: the next
+// tile's MMAs run while the epilogue drains the previous one.  The backbone runs as a dense MMA over zero-filled codes:
 // the FP4 sparse MMA carries one scale per 32 logical elements, which cannot
 // express NVFP4's per-16 backbone scales.
 //
-// CTA layout (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
-// and MMA issuer, warps 2..5 = epilogue (one TMEM lane quarter each).
+// CTA layout (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
+// and MMA issuer, warps 2..5 = epilogue (one TMEM lane quarter each),
+// warps 6..9 = scale warps (block scales from shared into tensor memory).
 // Tile 128 x 128 x 256 (K in elements), 4-stage mbarrier pipeline; one
 // persistent CTA per SM walks the output tiles.
 #include "common.cuh"
@@ -50,8 +55,8 @@ struct alignas(8) Barriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];      // MMAs done (tcgen05.commit) + scale warps done reading
     uint64_t sf_full[kStages];    // scale factors of the stage are in tensor memory
-    uint64_t acc_full;      // MMAs of the current tile done (tcgen05.commit)
-    uint64_t acc_empty;     // epilogue has drained the accumulators (4 warps)
+    uint64_t acc_full[2];   // MMAs of a tile done (tcgen05.commit), per accumulator buffer
+    uint64_t acc_empty[2];  // epilogue has drained that buffer (4 warps)
     uint32_t tmem_base;
 };
 
@@ -198,7 +203,7 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
 // thread waits only until the epilogue has copied the previous tile's two
 // accumulators out of tensor memory, so the epilogue's global stores overlap
 // the next tile's MMAs.
-template <int FMT>
+template <int FMT, bool ONE>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_r,
               const __grid_constant__ CUtensorMap tm_w, const uint8_t* __restrict__ sf_b,
@@ -223,8 +228,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             mbar_init(&bars->empty[s], 1 + 4);
             mbar_init(&bars->sf_full[s], 4);
         }
-        mbar_init(&bars->acc_full, 1);
-        mbar_init(&bars->acc_empty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->acc_full[b], 1);
+            mbar_init(&bars->acc_empty[b], 4);
+        }
         fence_barrier_init();
     }
     if (warp == 1) { tmem_alloc(&bars->tmem_base, kTmemCols); tmem_relinquish(); }
@@ -273,9 +280,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             uint32_t it = 0, tc = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
-                // the epilogue must have drained the previous tile's accumulators
-                if (tc > 0 && !mbar_wait(&bars->acc_empty, (tc - 1) & 1)) { ok = false; break; }
+                // the epilogue must have drained this buffer's previous tile
+                const uint32_t buf = ONE ? (tc & 1u) : 0u;
+                const uint32_t use = ONE ? (tc >> 1) : tc;
+                if (use > 0 && !mbar_wait(&bars->acc_empty[buf], (use - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t d_b = ONE ? tmem + buf * BN : t_acc_b;
+                const uint32_t d_r = ONE ? d_b : t_acc_r;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
@@ -294,14 +305,14 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                         const uint32_t col = 4 * at;
                         const uint64_t db = sdesc_sw128(a_w + 32 * j);
                         const uint32_t acc = (kb | j) ? 1u : 0u;
-                        mma<FMT>(t_acc_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + col,
+                        mma<FMT>(d_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + col,
                                  acc, sf_id);
-                        mma<FMT>(t_acc_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + col,
-                                 acc, sf_id);
+                        mma<FMT>(d_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + col,
+                                 ONE ? 1u : acc, sf_id);
                     }
                     tc_commit(&bars->empty[s]);
                 }
-                tc_commit(&bars->acc_full);
+                tc_commit(&bars->acc_full[buf]);
             }
         }
     } else if (warp >= 6) {
@@ -316,12 +327,17 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
                 const uint8_t* sf = smem + s * C::kStageStride + 3 * kTileBytes;
                 const uint32_t tcol = tmem + 2 * BN + s * kSfColsPerStage + lane_off;
+                // one store per operand: its kAtoms atoms are 4 * kAtoms
+                // consecutive columns
 #pragma unroll
-                for (int o = 0; o < 3; ++o)
+                for (int o = 0; o < 3; ++o) {
+                    uint4 v[C::kAtoms];
 #pragma unroll
                     for (int at = 0; at < C::kAtoms; ++at)
-                        tmem_st_32x32b_x4(tcol + o * 4 * C::kAtoms + 4 * at,
-                                          ld_shared_v4(sf + o * C::kSfBytes + 512 * at + 16 * lane));
+                        v[at] = ld_shared_v4(sf + o * C::kSfBytes + 512 * at + 16 * lane);
+                    if constexpr (C::kAtoms == 4) tmem_st_32x32b_x16(tcol + o * 4 * C::kAtoms, v);
+                    else                          tmem_st_32x32b_x8(tcol + o * 4 * C::kAtoms, v);
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -341,33 +357,36 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             const int r_local = q * 32 + lane;
             const int64_t row = ti.y_row + r_local;
             const bool row_ok = r_local < ti.rows;
-            const bool ok = mbar_wait(&bars->acc_full, tc & 1);
+            const uint32_t buf = ONE ? (tc & 1u) : 0u;
+            const uint32_t use = ONE ? (tc >> 1) : tc;
+            const bool ok = mbar_wait(&bars->acc_full[buf], use & 1);
             tc_fence_after();
             if (!ok) break;
+            const uint32_t src_b = ONE ? tmem + buf * BN : t_acc_b;
             const int64_t col0 = ti.col;
             if (ep.y_fp32) {
 #pragma unroll 1
                 for (int cc = 0; cc < BN / 32; ++cc) {
                     uint32_t vb[32], vr[32];
-                    tmem_ld_32x32b_x32(t_acc_b + lane_off + cc * 32, vb);
-                    tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
+                    tmem_ld_32x32b_x32(src_b + lane_off + cc * 32, vb);
+                    if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
                     tmem_ld_wait();
                     if (row_ok) {
                         float* y = static_cast<float*>(ep.Y) + row * ep.N + col0 + cc * 32;
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {
-                            float4 o;
-                            o.x = gb * __uint_as_float(vb[i + 0]) + gr * __uint_as_float(vr[i + 0]);
-                            o.y = gb * __uint_as_float(vb[i + 1]) + gr * __uint_as_float(vr[i + 1]);
-                            o.z = gb * __uint_as_float(vb[i + 2]) + gr * __uint_as_float(vr[i + 2]);
-                            o.w = gb * __uint_as_float(vb[i + 3]) + gr * __uint_as_float(vr[i + 3]);
-                            *reinterpret_cast<float4*>(y + i) = o;
+                            float o[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                o[u] = ONE ? gb * __uint_as_float(vb[i + u])
+                                           : gb * __uint_as_float(vb[i + u]) + gr * __uint_as_float(vr[i + u]);
+                            *reinterpret_cast<float4*>(y + i) = make_float4(o[0], o[1], o[2], o[3]);
                         }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->acc_empty);
+                if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
             } else {
                 // drain both accumulators into 64 packed bf16x2 registers, hand
                 // the tensor memory back, then store
@@ -375,20 +394,22 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
 #pragma unroll
                 for (int cc = 0; cc < BN / 32; ++cc) {
                     uint32_t vb[32], vr[32];
-                    tmem_ld_32x32b_x32(t_acc_b + lane_off + cc * 32, vb);
-                    tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
+                    tmem_ld_32x32b_x32(src_b + lane_off + cc * 32, vb);
+                    if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
                     tmem_ld_wait();
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {
-                        float lo = gb * __uint_as_float(vb[2 * h]) + gr * __uint_as_float(vr[2 * h]);
-                        float hi = gb * __uint_as_float(vb[2 * h + 1]) + gr * __uint_as_float(vr[2 * h + 1]);
+                        float lo = ONE ? gb * __uint_as_float(vb[2 * h])
+                                       : gb * __uint_as_float(vb[2 * h]) + gr * __uint_as_float(vr[2 * h]);
+                        float hi = ONE ? gb * __uint_as_float(vb[2 * h + 1])
+                                       : gb * __uint_as_float(vb[2 * h + 1]) + gr * __uint_as_float(vr[2 * h + 1]);
                         __nv_bfloat162 p2 = __floats2bfloat162_rn(lo, hi);
                         out[cc * 16 + h] = *reinterpret_cast<uint32_t*>(&p2);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->acc_empty);
+                if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
                 if (sc.grouped) {
                     // rows past the group belong to the next expert: masked row stores
                     if (row_ok) {
@@ -469,13 +490,13 @@ size_t linear_smem_bytes() {
     return kStages * Cfg<FMT>::kStageStride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
 }
 
-template <int FMT>
+template <int FMT, bool ONE>
 cudaError_t ensure_smem_attr() {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(linear_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(linear_kernel<FMT, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)linear_smem_bytes<FMT>());
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_set[dev] = true;
@@ -485,8 +506,8 @@ cudaError_t ensure_smem_attr() {
 
 // A_rows: rows of the activation operands (gathered and padded for the
 // grouped form); W_rows: rows of the (stacked) weight.
-template <int FMT>
-cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void* rs_codes,
+template <int FMT, bool ONE>
+cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const void* rs_codes,
                         const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
                         const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
     CUtensorMap tb, tr, tw;
@@ -494,14 +515,24 @@ cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void*
         !make_code_map(&tr, rs_codes, A_rows, p.K / 2, BM) ||
         !make_code_map(&tw, p.w_codes, W_rows, p.K / 2, BN))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr<FMT>();
+    cudaError_t e = ensure_smem_attr<FMT, ONE>();
     if (e != cudaSuccess) return e;
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
     const int grid = std::max(1, std::min(max_tiles, std::max(1, sms)));
-    linear_kernel<FMT><<<grid, kThreads, linear_smem_bytes<FMT>(), s>>>(
+    linear_kernel<FMT, ONE><<<grid, kThreads, linear_smem_bytes<FMT>(), s>>>(
         tb, tr, tw, static_cast<const uint8_t*>(bb_scales), static_cast<const uint8_t*>(rs_scales),
         static_cast<const uint8_t*>(p.w_scales), p.K, ep, sc);
     return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void* rs_codes,
+                        const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
+                        const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
+    return p.one_acc ? launch_gemm_t<FMT, true>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows, p,
+                                               W_rows, sc, max_tiles, s, sms)
+                     : launch_gemm_t<FMT, false>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows, p,
+                                                W_rows, sc, max_tiles, s, sms);
 }
 
 template <int FMT>

@@ -59,6 +59,8 @@ extern "C" SHARQ_API sharq_status sharq_prepare_noalloc(const void* X_bf16, cons
     if (!(o.fmt == SHARQ_NVFP4 || o.fmt == SHARQ_MXFP4) || o.K <= 0 || o.K % 256 != 0)
         return SHARQ_ERR_INVALID_ARG;
     if (!(o.m == 2 || o.m == 4 || o.m == 8) || o.n < 1 || o.n > o.m) return SHARQ_ERR_INVALID_ARG;
+    if (o.residual_scale != SHARQ_RESIDUAL_OWN && o.residual_scale != SHARQ_RESIDUAL_SHARED)
+        return SHARQ_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !(eps < 1e30f)) return SHARQ_ERR_INVALID_ARG;
     if (!o.bb_tscale || !o.rs_tscale) return SHARQ_ERR_INVALID_ARG;
     if (o.M > 0 && (!X_bf16 || !o.bb_codes || !o.bb_scales || !o.rs_codes || !o.rs_scales))
@@ -72,7 +74,7 @@ extern "C" SHARQ_API sharq_status sharq_prepare_noalloc(const void* X_bf16, cons
     if (!scratch) return SHARQ_ERR_CUDA;
     sharq::PrepareLaunch p{};
     p.X = X_bf16; p.gamma = gamma_bf16; p.eps = eps; p.M = o.M; p.K = o.K; p.n = o.n; p.m = o.m;
-    p.fmt = o.fmt; p.weight = false;
+    p.fmt = o.fmt; p.weight = false; p.residual_shared = o.residual_scale == SHARQ_RESIDUAL_SHARED;
     p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
     p.rs_codes = o.rs_codes; p.rs_scales = o.rs_scales; p.rs_tscale = o.rs_tscale;
     p.mask = o.mask;

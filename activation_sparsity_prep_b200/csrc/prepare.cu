@@ -290,9 +290,11 @@ struct LaneBlock {
 
 // ------------------------------------------------------------------------
 // The kernel.  FMT: 0 NVFP4, 1 MXFP4.  WEIGHT: quantise the whole tensor
-// once (keep-all, no norm, no residual).  NM24: the 2-of-4 mask.
+// once (keep-all, no norm, no residual).  NM24: the 2-of-4 mask.  RS: the
+// residual takes the backbone's tensor scale (NVFP4), so it is finished in
+// phase 2 with the backbone's reciprocal table and phase 3 does not exist.
 // ------------------------------------------------------------------------
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS>
 __global__ void __launch_bounds__(kThreads, 2)
 prepare_kernel(PrepArgs a) {
     __shared__ float s_inv[128];
@@ -403,7 +405,10 @@ prepare_kernel(PrepArgs a) {
     if (FMT == 0) {
         sb = nv_scale(__uint_as_float(ld_acquire_gpu(&a.ws[0])));
         fill_inv_table(s_inv, sb.genc);
-        if (blockIdx.x == 0 && threadIdx.x == 0) *a.bb_tscale = sb.gdec;
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            *a.bb_tscale = sb.gdec;
+            if (RS) *a.rs_tscale = sb.gdec;
+        }
     } else {
         if (blockIdx.x == 0 && threadIdx.x == 0) {
             *a.bb_tscale = 1.0f;
@@ -483,7 +488,21 @@ prepare_kernel(PrepArgs a) {
 #pragma unroll
                     for (int t = 0; t < 8; ++t) y[8 * v + t] = __fsub_rn(y[8 * v + t], d[t]);
                 }
-                if (FMT == 0) {
+                if (FMT == 0 && RS) {
+                    // the residual's block scale against the backbone's G
+                    const uint32_t er = cvt_e4m3(__fmul_rn(amaxE<E>(y), sb.k1));
+                    const float inv_r = s_inv[er];
+                    uint32_t rc[E / 8];
+#pragma unroll
+                    for (int v = 0; v < E / 8; ++v) {
+                        float t8[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[8 * v + t], inv_r);
+                        rc[v] = cvt_e2m1x8(t8);
+                    }
+                    *reinterpret_cast<uint2*>(a.rs_codes + row * (K / 2) + (int64_t)cb * 8) = make_uint2(rc[0], rc[1]);
+                    a.rs_scales[sf_off(row, cb, nsf)] = (uint8_t)er;
+                } else if (FMT == 0) {
                     ramax = fmaxf(ramax, amaxE<E>(y));
                 } else {
                     // MXFP4: the residual needs no tensor-wide scale; finish it here.
@@ -506,7 +525,7 @@ prepare_kernel(PrepArgs a) {
             lb = ln;
         }
     }
-    if (FMT == 1 || WEIGHT) return;
+    if (FMT == 1 || WEIGHT || RS) return;
 
     block_amax_to_global(ramax, &a.ws[1], s_red);
     grid_barrier(&a.ws[2], 2u * gridDim.x);
@@ -569,9 +588,9 @@ prepare_kernel(PrepArgs a) {
     }
 }
 
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
-    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24>;
+    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS>;
     static int blocks_per_sm = 0;          // same for every device of one architecture
     if (blocks_per_sm == 0) {
         int b = 0;
@@ -599,13 +618,13 @@ cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     return cudaLaunchKernelEx(&cfg, kfn, a);
 }
 
-template <int FMT, bool HAS_GAMMA, bool WEIGHT>
+template <int FMT, bool HAS_GAMMA, bool WEIGHT, bool RS = false>
 cudaError_t launch_m(const PrepArgs& a, int m, cudaStream_t s, int sms) {
     switch (m) {
-        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false>(a, s, sms);
-        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true>(a, s, sms)
-                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false>(a, s, sms);
-        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false>(a, s, sms);
+        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false, RS>(a, s, sms);
+        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true, RS>(a, s, sms)
+                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false, RS>(a, s, sms);
+        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false, RS>(a, s, sms);
     }
 }
 
@@ -639,6 +658,8 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
         return p.fmt == 0 ? launch_one<0, false, 8, true, false>(a, s, sms)
                           : launch_one<1, false, 8, true, false>(a, s, sms);
     }
+    if (p.fmt == 0 && p.residual_shared)
+        return g ? launch_m<0, true, false, true>(a, p.m, s, sms) : launch_m<0, false, false, true>(a, p.m, s, sms);
     if (p.fmt == 0) return g ? launch_m<0, true, false>(a, p.m, s, sms) : launch_m<0, false, false>(a, p.m, s, sms);
     return g ? launch_m<1, true, false>(a, p.m, s, sms) : launch_m<1, false, false>(a, p.m, s, sms);
 }

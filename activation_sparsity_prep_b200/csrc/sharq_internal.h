@@ -17,6 +17,7 @@ struct PrepareLaunch {
     int64_t M;
     int K, n, m, fmt;
     bool weight;          // quantise a whole weight tensor (keep-all, no residual)
+    bool residual_shared; // NVFP4 residual quantised with the backbone's tensor scale
     void* bb_codes;
     void* bb_scales;
     float* bb_tscale;
@@ -44,6 +45,7 @@ struct LinearLaunch {
     int N, K, fmt;
     void* Y;
     int y_fp32;
+    bool one_acc;             // G_b == G_r: both paths into one accumulator
     // grouped form
     const int32_t* row_index; // may be null
     const int32_t* offsets;   // null for the plain linear

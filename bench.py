@@ -53,6 +53,8 @@ def parse_args():
                     help="rows per linear (default: 2048 for llama8b, the workload's own M otherwise)")
     ap.add_argument("--fmt", default="nvfp4")
     ap.add_argument("--nm", default="2:4", help="n:m of the backbone mask")
+    ap.add_argument("--residual", choices=["own", "shared"], default="own",
+                    help="tensor scale of the NVFP4 residual: its own (default) or the backbone's")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -272,7 +274,7 @@ def build_units(args, dev):
             Wt = up(d["W"])
             w = sq.quantize_weight(Wt, fmt)
             del Wt
-            P = sq.Prepared.empty(M, L.K, n, m, fmt, device=dev)
+            P = sq.Prepared.empty(M, L.K, n, m, fmt, device=dev, residual_scale=args.residual)
             ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
             Y = torch.empty((M, L.N), dtype=bf, device=dev)
             u = dict(name=L.name, rows=M, prep_rows=M, N=L.N, K=L.K, X=X, Y=Y)
@@ -296,7 +298,7 @@ def build_units(args, dev):
             we = sq.Weight(w.codes[e], w.scales[e * sb:(e + 1) * sb], w.tensor_scale[e:e + 1],
                            L.N, L.K, w.fmt)
             sq.quantize_weight(up(wl.weight(W.cfg * 1000 + li, 100 + e, L.N, L.K)), fmt, out=we)
-        P = sq.Prepared.empty(rows_in, L.K, n, m, fmt, device=dev)
+        P = sq.Prepared.empty(rows_in, L.K, n, m, fmt, device=dev, residual_scale=args.residual)
         ws = torch.empty(max(256, sq.prepare_workspace_bytes(rows_in, L.K, fmt)), dtype=torch.uint8, device=dev)
         mws = torch.empty(sq.moe_workspace_bytes(T * topk, E, L.K, fmt), dtype=torch.uint8, device=dev)
         Y = torch.empty((T * topk, L.N), dtype=bf, device=dev)
@@ -459,6 +461,7 @@ def run_sharq(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4" if fmt == 0 else "mxfp4", "data": "synthetic",
             "config": {"workload": desc, "M": tokens_per_step, "fmt": args.fmt, "nm": args.nm,
+                       "residual_scale": args.residual,
                        "l2": "flushed between timed steps (512 MiB write)",
                        "timing": "CUDA graph per step, per-kernel external events"},
             "tokens_per_s": tokens,

@@ -70,6 +70,18 @@ typedef enum {
     SHARQ_MXFP4 = 1    /* E2M1 codes, E8M0 scale per 32 elements, no tensor scale   */
 } sharq_format;
 
+/* Tensor scale of the residual (NVFP4).  The abstract gives every FP4
+ * tensor its own scaling without saying whether the residual shares the
+ * backbone's; OWN (its own amax) is the plain reading and the default.
+ * SHARED quantises the residual against the backbone's tensor amax, so
+ * G_r = G_b: the preparation needs one tensor-wide reduction fewer and the
+ * linear accumulates both paths in one accumulator.  MXFP4 has no tensor
+ * scale, so the setting changes nothing there. */
+typedef enum {
+    SHARQ_RESIDUAL_OWN = 0,
+    SHARQ_RESIDUAL_SHARED = 1
+} sharq_residual_scale;
+
 /* One FP4 weight payload shared by both GEMM paths (Abstract: a single FP4
  * weight payload with path-specific scale views).  Both paths use the same
  * codes and the same MMA-ready scale atoms, which is the layout the block-
@@ -95,6 +107,7 @@ typedef struct {
     void*  mask;         /* optional [M, K/8] bitmask, NULL to skip         */
     int    M, K, n, m;
     int    fmt;          /* sharq_format */
+    int    residual_scale;   /* sharq_residual_scale (0 = OWN)              */
 } sharq_prepared;
 
 /* Human-readable name of a status code (static string). */
@@ -127,7 +140,8 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_wei
  *         (lower index first on ties);
  *   backbone B = keep ? y : 0, quantised to FP4 with its own tensor scale;
  *   residual r = y - dequant(Q(B)), quantised to FP4 with its own tensor
- *         scale.
+ *         scale (out->residual_scale = SHARQ_RESIDUAL_OWN) or the
+ *         backbone's (SHARQ_RESIDUAL_SHARED).
  * Fills the buffers named in *out (out->M, K, n, m, fmt must match the
  * arguments).  Supported: m in {2, 4, 8}, 1 <= n <= m.  ws:
  * sharq_prepare_workspace_bytes(M, K, fmt) bytes. */
@@ -140,7 +154,10 @@ SHARQ_API sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16,
  *   Y[i,j] = G_w * (G_b * S_b[i,j] + G_r * S_r[i,j]),
  *   S_p = sum_k val(p)[i,k] s(p)[i,k/B] * val(w)[j,k] s(w)[j,k/B].
  * Both products accumulate in fp32 tensor memory from one weight tile per
- * k-step.  Y is bf16 [M, N] (y_is_fp32 = 0) or fp32 [M, N]. */
+ * k-step, in two accumulators; when G_b = G_r by construction (MXFP4, whose
+ * tensor scales sharq_prepare writes as 1, or SHARQ_RESIDUAL_SHARED) in one,
+ * Y = G_w * G_b * (S_b + S_r), and rs_tscale is not read.  Y is bf16
+ * [M, N] (y_is_fp32 = 0) or fp32 [M, N]. */
 SHARQ_API sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w,
                           void* Y, int y_is_fp32, void* stream);
 

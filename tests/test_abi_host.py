@@ -41,12 +41,12 @@ def test_atom_layout_is_a_permutation():
     assert np.array_equal(np.sort(idx.ravel()), np.arange(256 * 64))
 
 
-def _fake_prepared(M=16, K=256, n=2, m=4, fmt=0, p=0x1000):
-    return sq._Prepared(p, p, p, p, p, p, None, M, K, n, m, fmt)
+def _fake_prepared(M=16, K=256, n=2, m=4, fmt=0, p=0x1000, rs=0):
+    return sq._Prepared(p, p, p, p, p, p, None, M, K, n, m, fmt, rs)
 
 
 @pytest.mark.parametrize("kw", [dict(K=100), dict(m=3), dict(n=0), dict(n=5), dict(fmt=7),
-                                dict(M=-1), dict(p=0x1001)])
+                                dict(M=-1), dict(p=0x1001), dict(rs=2), dict(rs=-1)])
 def test_prepare_rejects_bad_arguments_on_host(kw):
     L = sq.load_sharq_ops()
     cp = _fake_prepared(**kw)
@@ -89,3 +89,14 @@ def test_status_strings():
     L = sq.load_sharq_ops()
     assert L.sharq_status_string(0) == b"ok"
     assert L.sharq_status_string(4) == b"device wait timed out"
+
+
+def test_unknown_residual_scale_is_rejected_everywhere():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared(rs=3)
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 0)
+    assert L.sharq_linear(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0, None) == 1
+    ws = sq.moe_workspace_bytes(16, 4, 256)
+    assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000, 0,
+                              0x1000, ws, None) == 1
+    assert L.sharq_prepare_noalloc(0x1000, None, 1e-6, ctypes.byref(cp), None) == 1

@@ -3,9 +3,11 @@
 Tolerances:
 * fp32 output: relative Frobenius error <= 1e-5 against the fp64 result.
 * fp32 output, element by element: |Y32 - Y64| <= gamma * A with
-  A = G_w (G_b |Db||Dw|^T + G_r |Dr||Dw|^T) and gamma = (K/64 + 2) * 2^-23,
-  the recursive-summation bound for K/64 fp32 accumulations of exact 64-term
-  MMA partial sums, with a factor 2 for the tensor core's internal rounding.
+  A = G_w (G_b |Db||Dw|^T + G_r |Dr||Dw|^T) and gamma = (C + 2) * 2^-23,
+  the recursive-summation bound for C fp32 accumulations of exact 64-term
+  MMA partial sums, with a factor 2 for the tensor core's internal rounding:
+  C = K/64 when each path has its own accumulator, C = 2K/64 when both
+  paths share one (MXFP4, or a residual with the backbone's tensor scale).
 * bf16 output: within one bf16 ulp of RNE(Y64); where cancellation makes
   gamma * A larger than half an ulp (no fp32 accumulation can do better
   there), within one ulp plus gamma * A.  The number of such elements is
@@ -56,16 +58,16 @@ def bf16_ulp(v):
     return 2.0 ** (e - 7)
 
 
-def check(Y32, Ybf, Y64, A, K, rows=None):
+def check(Y32, Ybf, Y64, A, K, rows=None, one_acc=False):
     """Returns (relative Frobenius error, elements needing the widened bf16
-    tolerance)."""
+    tolerance).  one_acc: both paths were accumulated in one chain."""
     Y32 = to_np(Y32).astype(np.float64)
     got = to_np(Ybf)
     if rows is not None:
         Y32, got = Y32[rows], got[rows]
     err = np.linalg.norm(Y32 - Y64) / max(np.linalg.norm(Y64), 1e-300)
     assert err <= FROB_TOL, f"relative Frobenius error {err:.3e}"
-    gamma = (K / 64 + 2) * 2.0 ** -23
+    gamma = ((2 if one_acc else 1) * K / 64 + 2) * 2.0 ** -23
     bound = gamma * A + 2.0 ** -126
     e32 = np.abs(Y32 - Y64)
     assert np.all(e32 <= bound), f"fp32 error beyond the summation bound: max ratio {(e32 / bound).max():.2f}"
@@ -107,7 +109,7 @@ def test_linear_matches_oracle(M, N, K, fmt):
     Ybf = sq.linear(P, w)
     torch.cuda.synchronize()
     assert sq.last_device_status() == 0
-    check(Y32, Ybf, oracle.linear(R, Rw), oracle.linear_abs(R, Rw), K)
+    check(Y32, Ybf, oracle.linear(R, Rw), oracle.linear_abs(R, Rw), K, one_acc=fmt == "mxfp4")
 
 
 def test_linear_pipeline_through_gpu_prepare():
@@ -162,3 +164,30 @@ def test_linear_full_size_llama_prefill_sampled(lin):
     rows = np.sort(np.random.default_rng(lin).choice(2048, 48, replace=False))
     check(Y32, Ybf, oracle.linear(R, Rw, rows=rows), oracle.linear_abs(R, Rw, rows=rows), L.K,
           rows=rows)
+
+
+# ---------------------------------------------------------------------------
+# Residual with the backbone's tensor scale: one accumulator for both paths.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K,gk", [(16, 256, 256, "ones"), (300, 512, 4096, "ones"),
+                                      (129, 384, 1024, None), (2048, 1024, 4096, "random")])
+def test_linear_shared_residual_scale(M, N, K, gk):
+    """GPU prepare (shared) bit-exact against the oracle, then the
+    single-accumulator linear against the fp64 two-path product."""
+    X = wl.activation("laplace_outlier", 33, M + K, M, K)
+    g = None if gk is None else (wl.gamma_ones(K) if gk == "ones" else wl.gamma_random(33, 0, K))
+    W = wl.weight(33, N, N, K)
+    P = sq.prepare(to_dev(X), None if g is None else to_dev(g), wl.EPS, residual_scale="shared")
+    w = sq.quantize_weight(to_dev(W))
+    Y32 = sq.linear(P, w, out_fp32=True)
+    Ybf = sq.linear(P, w)
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    R = oracle.prepare(X, g, wl.EPS, residual_scale="shared")
+    Rw = oracle.quantize_weight(W)
+    assert np.array_equal(to_np(P.rs_codes), R.rs.codes)
+    assert to_np(P.rs_tscale).view(np.uint32)[0] == np.float32(R.rs.tscale).view(np.uint32)
+    rows = None if M <= 512 else np.sort(np.random.default_rng(M).choice(M, 48, replace=False))
+    check(Y32, Ybf, oracle.linear(R, Rw, rows=rows), oracle.linear_abs(R, Rw, rows=rows), K,
+          rows=rows, one_acc=True)

@@ -30,21 +30,21 @@ def dispatch(experts, E):
     return ri, off
 
 
-def run_case(T_tok, E, topk, K, N, experts=None, fmt="nvfp4", seed=51):
+def run_case(T_tok, E, topk, K, N, experts=None, fmt="nvfp4", seed=51, residual_scale="own"):
     X = wl.activation("laplace_outlier", seed, 0, T_tok, K)
     g = wl.gamma_ones(K)
     if experts is None:
         experts = wl.routing(seed, T_tok, E, topk)
     ri, off = dispatch(experts, E)
     Ws, w = stacked_weights(seed, E, N, K, fmt)
-    P = sq.prepare(to_dev(X), to_dev(g), wl.EPS, 2, 4, fmt)
+    P = sq.prepare(to_dev(X), to_dev(g), wl.EPS, 2, 4, fmt, residual_scale=residual_scale)
     ri_d = torch.from_numpy(ri).cuda()
     off_d = torch.from_numpy(off).cuda()
     Y32 = sq.moe_linear(P, ri_d, off_d, w, out_fp32=True)
     Ybf = sq.moe_linear(P, ri_d, off_d, w)
     torch.cuda.synchronize()
     assert sq.last_device_status() == 0
-    R = oracle.prepare(X, g, wl.EPS, 2, 4, fmt)
+    R = oracle.prepare(X, g, wl.EPS, 2, 4, fmt, residual_scale=residual_scale)
     Rws = [oracle.quantize_weight(W, fmt) for W in Ws]
     Y64 = oracle.moe_linear(R, ri, off, Rws)
     # the summation bound of every dispatched row, from its own expert
@@ -54,7 +54,7 @@ def run_case(T_tok, E, topk, K, N, experts=None, fmt="nvfp4", seed=51):
         idx = np.nonzero(grp == e)[0]
         if len(idx):
             A[idx] = oracle.linear_abs(oracle.gather_rows(R, ri[idx]), Rws[e])
-    return check(Y32, Ybf, Y64, A, K)
+    return check(Y32, Ybf, Y64, A, K, one_acc=fmt == "mxfp4" or residual_scale == "shared")
 
 
 def test_moe_small_uniform_routing():
@@ -72,6 +72,10 @@ def test_moe_uneven_and_empty_experts():
 
 def test_moe_mxfp4():
     run_case(T_tok=96, E=4, topk=2, K=256, N=128, fmt="mxfp4")
+
+
+def test_moe_shared_residual_scale():
+    run_case(T_tok=200, E=3, topk=2, K=512, N=256, residual_scale="shared")
 
 
 def test_moe_single_expert_equals_linear():

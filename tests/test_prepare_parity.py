@@ -21,12 +21,13 @@ def _gamma(kind, cfg, K):
     return None
 
 
-def run_and_compare(X, g, n, m, fmt, eps=1e-6):
+def run_and_compare(X, g, n, m, fmt, eps=1e-6, residual_scale="own"):
     M, K = X.shape
-    P = sq.prepare(to_dev(X), None if g is None else to_dev(g), eps, n, m, fmt, want_mask=True)
+    P = sq.prepare(to_dev(X), None if g is None else to_dev(g), eps, n, m, fmt, want_mask=True,
+                   residual_scale=residual_scale)
     torch.cuda.synchronize()
     assert sq.last_device_status() == 0
-    R = oracle.prepare(X, g, eps, n, m, fmt)
+    R = oracle.prepare(X, g, eps, n, m, fmt, residual_scale=residual_scale)
     assert np.array_equal(to_np(P.mask), R.mask), "mask"
     assert np.array_equal(to_np(P.bb_codes), R.bb.codes), "backbone codes"
     assert np.array_equal(to_np(P.rs_codes), R.rs.codes), "residual codes"
@@ -72,6 +73,23 @@ CASES = [
 def test_prepare_bit_exact(M, K, dist, gk, n, m, fmt):
     X = wl.activation(dist, 21, M + K, M, K)
     run_and_compare(X, _gamma(gk, 21, K), n, m, fmt)
+
+
+SHARED_CASES = [
+    # M, K, dist, gamma, n, m
+    (16, 256, "normal_outlier", "ones", 2, 4),
+    (3, 768, "laplace_outlier", None, 2, 4),
+    (129, 2048, "student_t", "random", 1, 4),
+    (300, 512, "laplace_outlier", "ones", 4, 8),
+    (700, 3584, "student_t", None, 2, 4),
+]
+
+
+@pytest.mark.parametrize("M,K,dist,gk,n,m", SHARED_CASES)
+def test_prepare_shared_residual_scale_bit_exact(M, K, dist, gk, n, m):
+    X = wl.activation(dist, 24, M + K, M, K)
+    P, R = run_and_compare(X, _gamma(gk, 24, K), n, m, "nvfp4", residual_scale="shared")
+    assert torch.equal(P.rs_tscale, P.bb_tscale)
 
 
 def test_prepare_special_values():
