@@ -73,8 +73,11 @@ def lib() -> ctypes.CDLL:
             L.orc_quant_nvfp4_amax.argtypes = [P, i64, i32, f32, P, P, P, P]
             L.orc_tensor_amax.argtypes = [P, i64]
             L.orc_tensor_amax.restype = f32
-            L.orc_prepare.argtypes = [P, P, f32, i64, i32, i32, i32, i32, i32,
+            L.orc_prepare.argtypes = [P, P, P, i32, f32, i64, i32, i32, i32, i32, i32,
                                       P, P, P, P, P, P, P, P, P]
+            L.orc_ln_stats.argtypes = [P, i32, f32, P, P]
+            L.orc_ln_stats.restype = i32
+            L.orc_normalize_ln.argtypes = [P, P, P, f32, i64, i32, P]
             L.orc_prepare.restype = i32
             L.orc_quantize_weight.argtypes = [P, i64, i32, i32, P, P, P]
             L.orc_quantize_weight.restype = i32
@@ -190,14 +193,36 @@ class Prepared:
 RESIDUAL_SCALES = {"own": 0, "shared": 1}
 
 
+def ln_stats(x: np.ndarray, eps: float = 1e-6):
+    """(mu, rstd) of one bf16 row under the LayerNorm reading."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    mu = np.zeros(1, dtype=np.float32)
+    rs = np.zeros(1, dtype=np.float32)
+    if lib().orc_ln_stats(_p(x), x.shape[-1], eps, _p(mu), _p(rs)) != 0:
+        raise ValueError("bad row")
+    return mu[0], rs[0]
+
+
+def normalize_ln(X: np.ndarray, gamma: np.ndarray, beta: Optional[np.ndarray], eps: float = 1e-6):
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    M, K = X.shape
+    y = np.empty((M, K), dtype=np.float32)
+    b = None if beta is None else np.ascontiguousarray(beta, dtype=np.uint16)
+    lib().orc_normalize_ln(_p(X), _p(np.ascontiguousarray(gamma, dtype=np.uint16)), _p(b), eps, M, K, _p(y))
+    return y
+
+
 def prepare(X: np.ndarray, gamma: Optional[np.ndarray], eps: float = 1e-6,
             n: int = 2, m: int = 4, fmt="nvfp4", keep_intermediates: bool = False,
-            residual_scale: str = "own") -> Prepared:
+            residual_scale: str = "own", norm: str = "rms",
+            beta: Optional[np.ndarray] = None) -> Prepared:
     """The preparation operator on a whole tensor X [M, K] (bf16 bits).
 
     residual_scale "own": the residual is quantised with its own tensor
     scale (the plain reading of the abstract); "shared": with the backbone's
-    (NVFP4 only; MXFP4 has no tensor scale, so both settings agree)."""
+    (NVFP4 only; MXFP4 has no tensor scale, so both settings agree).
+    norm "rms": RMSNorm with gamma (no norm when gamma is None); "layernorm":
+    LayerNorm with gamma and an optional beta."""
     fmt = _fmt(fmt)
     X = np.ascontiguousarray(X, dtype=np.uint16)
     M, K = X.shape
@@ -212,7 +237,10 @@ def prepare(X: np.ndarray, gamma: Optional[np.ndarray], eps: float = 1e-6,
     rg = np.zeros(1, dtype=np.float32)
     y = np.empty((M, K), dtype=np.float32) if keep_intermediates else None
     r = np.empty((M, K), dtype=np.float32) if keep_intermediates else None
-    rc_ = lib().orc_prepare(_p(X), _p(g), eps, M, K, n, m, fmt,
+    if norm not in ("rms", "layernorm"):
+        raise ValueError(norm)
+    b = None if beta is None else np.ascontiguousarray(beta, dtype=np.uint16)
+    rc_ = lib().orc_prepare(_p(X), _p(g), _p(b), int(norm == "layernorm"), eps, M, K, n, m, fmt,
                             RESIDUAL_SCALES[residual_scale], _p(mk),
                             _p(bc), _p(bs), _p(bg), _p(rc), _p(rsc), _p(rg),
                             _p(y), _p(r))

@@ -175,6 +175,67 @@ static inline float bf16f(uint16_t b) {
     uint32_t u = (uint32_t)b << 16; float f; memcpy(&f, &u, 4); return f;
 }
 
+/* ------------------------------------------------------------------------ */
+/* LayerNorm statistics (the mean-subtracting norm of DiT and vision         */
+/* layers, which the pages name among the evaluated models; the reading of   */
+/* its precision is this library's):                                         */
+/*   S1 = sum x_k and S2 = sum (x_k - mu)^2, each in the canonical order of  */
+/*   the RMS sum above (32 lanes, chunk c to lane c mod 32, element order    */
+/*   inside a lane, xor butterfly 16..1);                                    */
+/*   mu = S1 / K;  d_k = x_k - mu;  var = S2 / K;                            */
+/*   rstd = 1 / sqrt(var + eps);  y_k = (d_k * rstd) * gamma_k [+ beta_k].   */
+/* Two passes (mean, then centred squares): the textbook stable form.        */
+/* Pinned: constant row (y = beta exactly), a +-a row against its closed     */
+/* form, and a lane-order probe on S1.                                       */
+/* ------------------------------------------------------------------------ */
+
+static float canonical_sum(const float* v, int K) {
+    float lane[32];
+    for (int l = 0; l < 32; ++l) lane[l] = 0.0f;
+    for (int c = 0; c < K / 8; ++c)
+        for (int t = 0; t < 8; ++t) lane[c % 32] = lane[c % 32] + v[8 * c + t];
+    for (int o = 16; o >= 1; o >>= 1) {
+        float nxt[32];
+        for (int l = 0; l < 32; ++l) nxt[l] = lane[l] + lane[l ^ o];
+        memcpy(lane, nxt, sizeof(lane));
+    }
+    return lane[0];
+}
+
+/* mu and rstd of one row; returns -1 if K is not a multiple of 8 or too big */
+int orc_ln_stats(const uint16_t* x_bf16, int K, float eps, float* mu_out, float* rstd_out) {
+    if (K <= 0 || K % 8 != 0 || K > (1 << 20)) return -1;
+    float* v = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!v) return -1;
+    for (int k = 0; k < K; ++k) v[k] = bf16f(x_bf16[k]);
+    float mu = canonical_sum(v, K) / (float)K;
+    for (int k = 0; k < K; ++k) {
+        float d = v[k] - mu;
+        v[k] = d * d;
+    }
+    float var = canonical_sum(v, K) / (float)K;
+    float den = sqrtf(var + eps);
+    *mu_out = mu;
+    *rstd_out = 1.0f / den;
+    free(v);
+    return 0;
+}
+
+void orc_normalize_ln(const uint16_t* X, const uint16_t* gamma, const uint16_t* beta, float eps,
+                      int64_t M, int K, float* y) {
+    for (int64_t i = 0; i < M; ++i) {
+        const uint16_t* xr = X + i * (int64_t)K;
+        float* yr = y + i * (int64_t)K;
+        float mu = 0.0f, rstd = 1.0f;
+        orc_ln_stats(xr, K, eps, &mu, &rstd);
+        for (int k = 0; k < K; ++k) {
+            float d = bf16f(xr[k]) - mu;
+            float t = (d * rstd) * bf16f(gamma[k]);
+            yr[k] = beta ? t + bf16f(beta[k]) : t;
+        }
+    }
+}
+
 /* y = RMSNorm(x) * gamma per row, or y = x when gamma is NULL. */
 void orc_normalize(const uint16_t* X, const uint16_t* gamma, float eps,
                    int64_t M, int K, float* y) {
@@ -321,7 +382,8 @@ static void quant(int fmt, const float* T, int64_t R, int K,
 /* ------------------------------------------------------------------------ */
 /* Preparation operator (Abstract: norm + mask + backbone FP4 + residual     */
 /* against the dequantised backbone + residual FP4, one operator):           */
-/*   y = norm(x); keep = mask(y); B = keep ? y : +0;                         */
+/*   y = norm(x) (RMSNorm with gamma, none without, or LayerNorm with gamma  */
+/*       and an optional beta); keep = mask(y); B = keep ? y : +0;           */
 /*   (codes_b, scales_b, G_b, D_b) = Q(B); r = y - D_b;                      */
 /*   (codes_r, scales_r, G_r) = Q(r)   -- residual has its own tensor scale, */
 /*   or, with residual_shared (NVFP4), the backbone's: Q(r) is taken with    */
@@ -332,13 +394,14 @@ static void quant(int fmt, const float* T, int64_t R, int K,
 /* Returns 0, or -1 on a bad argument or allocation failure.                 */
 /* ------------------------------------------------------------------------ */
 
-int orc_prepare(const uint16_t* X, const uint16_t* gamma, float eps,
-                int64_t M, int K, int n, int m, int fmt, int residual_shared,
+int orc_prepare(const uint16_t* X, const uint16_t* gamma, const uint16_t* beta, int layernorm,
+                float eps, int64_t M, int K, int n, int m, int fmt, int residual_shared,
                 uint8_t* mask_bits,
                 uint8_t* bb_codes, uint8_t* bb_scales, float* bb_g,
                 uint8_t* rs_codes, uint8_t* rs_scales, float* rs_g,
                 float* y_out, float* r_out) {
     if (K <= 0 || m <= 0 || n < 0 || n > m || K % m != 0 || K % 32 != 0) return -1;
+    if (layernorm && !gamma) return -1;
     int64_t E = M * (int64_t)K;
     float* y = y_out ? y_out : (float*)malloc(sizeof(float) * (size_t)(E ? E : 1));
     float* B = (float*)malloc(sizeof(float) * (size_t)(E ? E : 1));
@@ -346,7 +409,8 @@ int orc_prepare(const uint16_t* X, const uint16_t* gamma, float eps,
     uint8_t* keep = (uint8_t*)malloc((size_t)(E ? E : 1));
     if (!y || !B || !D || !keep) { free(B); free(D); free(keep); if (!y_out) free(y); return -1; }
 
-    orc_normalize(X, gamma, eps, M, K, y);
+    if (layernorm) orc_normalize_ln(X, gamma, beta, eps, M, K, y);
+    else           orc_normalize(X, gamma, eps, M, K, y);
     orc_mask(y, M, K, n, m, keep);
     for (int64_t i = 0; i < E; ++i) B[i] = keep[i] ? y[i] : 0.0f;
     const float A_b = orc_tensor_amax(B, E);
