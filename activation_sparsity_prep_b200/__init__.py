@@ -85,6 +85,8 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_quantize_weight.restype = I
         L.sharq_prepare.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P, SZ, P]
         L.sharq_prepare.restype = I
+        L.sharq_prepare_layernorm.argtypes = [P, P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P, SZ, P]
+        L.sharq_prepare_layernorm.restype = I
         L.sharq_linear.argtypes = [ctypes.POINTER(_Prepared), ctypes.POINTER(_Weight), P, I, P]
         L.sharq_linear.restype = I
         L.sharq_moe_workspace_bytes.argtypes = [I64, I, I, I]
@@ -236,6 +238,24 @@ def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4
     _check("sharq_prepare",
            L.sharq_prepare(X.data_ptr(), _ptr(gamma), float(eps), ctypes.byref(cp),
                            ws.data_ptr(), ws.numel(), _stream(stream)))
+    return p
+
+
+def prepare_layernorm(X, gamma, beta=None, eps: float = 1e-6, n: int = 2, m: int = 4,
+                      fmt="nvfp4", want_mask: bool = False, out: Optional[Prepared] = None,
+                      ws=None, stream=None, residual_scale="own") -> Prepared:
+    """prepare() with LayerNorm (gamma required, beta optional) instead of
+    RMSNorm in front of the mask."""
+    L = load_sharq_ops()
+    M, K = X.shape
+    f = _fmt(fmt)
+    p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
+                                                   residual_scale=residual_scale)
+    ws = _workspace(M, K, f, ws, X.device)
+    cp = p._c()
+    _check("sharq_prepare_layernorm",
+           L.sharq_prepare_layernorm(X.data_ptr(), _ptr(gamma), _ptr(beta), float(eps),
+                                     ctypes.byref(cp), ws.data_ptr(), ws.numel(), _stream(stream)))
     return p
 
 

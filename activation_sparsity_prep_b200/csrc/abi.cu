@@ -86,9 +86,12 @@ sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_weight* out, 
                                              sharq::device_sm_count()));
 }
 
-sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps,
-                           const sharq_prepared* out, void* ws, size_t ws_bytes, void* stream) {
+static sharq_status prepare_common(const void* X_bf16, const void* gamma_bf16, const void* beta_bf16,
+                                   bool layernorm, float eps, const sharq_prepared* out, void* ws,
+                                   size_t ws_bytes, void* stream) {
     if (!out || !ws) return SHARQ_ERR_INVALID_ARG;
+    if (layernorm && out->M > 0 && !gamma_bf16) return SHARQ_ERR_INVALID_ARG;
+    if (!aligned16(beta_bf16)) return SHARQ_ERR_INVALID_ARG;
     const sharq_prepared& o = *out;
     if (!valid_fmt(o.fmt) || !valid_shape(o.M, o.K)) return SHARQ_ERR_INVALID_ARG;
     if (!(o.m == 2 || o.m == 4 || o.m == 8) || o.n < 1 || o.n > o.m) return SHARQ_ERR_INVALID_ARG;
@@ -106,12 +109,24 @@ sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps
     if (ws_bytes < sharq::prepare_ws_bytes(o.M)) return SHARQ_ERR_INVALID_ARG;
     sharq::PrepareLaunch p{};
     p.X = X_bf16; p.gamma = gamma_bf16; p.eps = eps; p.M = o.M; p.K = o.K; p.n = o.n; p.m = o.m;
+    p.beta = layernorm ? beta_bf16 : nullptr; p.layernorm = layernorm;
     p.fmt = o.fmt; p.weight = false; p.residual_shared = o.residual_scale == SHARQ_RESIDUAL_SHARED;
     p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
     p.rs_codes = o.rs_codes; p.rs_scales = o.rs_scales; p.rs_tscale = o.rs_tscale;
     p.mask = o.mask; p.ws = ws;
     return cuda_status(sharq::launch_prepare(p, static_cast<cudaStream_t>(stream),
                                              sharq::device_sm_count()));
+}
+
+sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps,
+                           const sharq_prepared* out, void* ws, size_t ws_bytes, void* stream) {
+    return prepare_common(X_bf16, gamma_bf16, nullptr, false, eps, out, ws, ws_bytes, stream);
+}
+
+sharq_status sharq_prepare_layernorm(const void* X_bf16, const void* gamma_bf16, const void* beta_bf16,
+                                     float eps, const sharq_prepared* out, void* ws, size_t ws_bytes,
+                                     void* stream) {
+    return prepare_common(X_bf16, gamma_bf16, beta_bf16, true, eps, out, ws, ws_bytes, stream);
 }
 
 static sharq_status check_linear_args(const sharq_prepared* x, const sharq_weight* w, void* Y) {

@@ -4,7 +4,8 @@
 // input-adaptive N:M mask, the FP4 backbone, and the residual taken against
 // the *dequantised* backbone.  The NVFP4 tensor scales make this a chain of
 // three tensor-wide dependencies:
-//   phase 1  rinv per row (RMSNorm) and A_b = max|y|      -> grid barrier
+//   phase 1  rinv per row (RMSNorm; LayerNorm: mean and rstd) and
+//            A_b = max|y|                                 -> grid barrier
 //   phase 2  mask, backbone codes/scales with G_b, residual r,
 //            A_r = max|r|                                 -> grid barrier
 //   phase 3  residual codes/scales with G_r
@@ -35,6 +36,7 @@ constexpr int kWarps = kThreads / 32;
 struct PrepArgs {
     const uint16_t* X;       // [M, K] bf16
     const uint16_t* gamma;   // [K] bf16 or null
+    const uint16_t* beta;    // [K] bf16 or null (LayerNorm bias)
     float eps;
     int64_t M;
     int K;
@@ -46,11 +48,16 @@ struct PrepArgs {
     uint8_t* rs_scales;
     float* rs_tscale;
     uint8_t* mask;           // optional
-    uint32_t* ws;            // [0] amax_b bits, [1] amax_r bits, [2] barrier, then rinv[M]
+    uint32_t* ws;            // [0] amax_b bits, [1] amax_r bits, [2] barrier, then rinv[M], mu[M]
 };
 
 __device__ __forceinline__ float* ws_rinv(uint32_t* ws) {
     return reinterpret_cast<float*>(ws + 16);
+}
+
+// LayerNorm means follow the M per-row reciprocals.
+__device__ __forceinline__ float* ws_mu(uint32_t* ws, int64_t M) {
+    return reinterpret_cast<float*>(ws + 16) + M;
 }
 
 // Byte offset of scale (row, s) in the MMA-ready atom layout.
@@ -255,13 +262,14 @@ __device__ __forceinline__ float amaxE(const float* v) {
     return m;
 }
 
-template <int FMT, bool HAS_GAMMA>
+template <int FMT, bool HAS_GAMMA, bool LN>
 struct LaneBlock {
     static constexpr int E = FMT == 0 ? 16 : 32;   // elements per lane = one scale block
     static constexpr int NV = E / 8;                // 16-byte chunks
     uint4 x[NV];
     uint4 g[NV];
-    float rinv;
+    uint4 b[LN ? NV : 1];
+    float rinv, mu;
 
     __device__ __forceinline__ void load(const PrepArgs& a, int64_t row, int cb, const float* rinv_ws) {
         const uint16_t* xp = a.X + row * a.K + (int64_t)cb * E;
@@ -272,9 +280,18 @@ struct LaneBlock {
             for (int v = 0; v < NV; ++v) g[v] = ld_nc_v4(a.gamma + (int64_t)cb * E + 8 * v);
             rinv = rinv_ws[row];
         }
+        if (LN) {
+            mu = rinv_ws[a.M + row];
+            if (a.beta) {
+#pragma unroll
+                for (int v = 0; v < NV; ++v) b[v] = ld_nc_v4(a.beta + (int64_t)cb * E + 8 * v);
+            }
+        }
     }
 
-    __device__ __forceinline__ void y(float* out) const {
+    // RMSNorm: fl(fl(x * rinv) * g).  LayerNorm: fl(fl(fl(x - mu) * rstd) * g),
+    // then + beta when there is a bias.
+    __device__ __forceinline__ void y(float* out, bool has_beta) const {
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
             unpack_bf16x8(x[v], out + 8 * v);
@@ -282,7 +299,16 @@ struct LaneBlock {
                 float gg[8];
                 unpack_bf16x8(g[v], gg);
 #pragma unroll
-                for (int t = 0; t < 8; ++t) out[8 * v + t] = __fmul_rn(__fmul_rn(out[8 * v + t], rinv), gg[t]);
+                for (int t = 0; t < 8; ++t) {
+                    const float xv = LN ? __fsub_rn(out[8 * v + t], mu) : out[8 * v + t];
+                    out[8 * v + t] = __fmul_rn(__fmul_rn(xv, rinv), gg[t]);
+                }
+                if (LN && has_beta) {
+                    float bb[8];
+                    unpack_bf16x8(b[v], bb);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) out[8 * v + t] = __fadd_rn(out[8 * v + t], bb[t]);
+                }
             }
         }
     }
@@ -294,12 +320,14 @@ struct LaneBlock {
 // residual takes the backbone's tensor scale (NVFP4), so it is finished in
 // phase 2 with the backbone's reciprocal table and phase 3 does not exist.
 // ------------------------------------------------------------------------
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS, bool LN>
 __global__ void __launch_bounds__(kThreads, 2)
 prepare_kernel(PrepArgs a) {
     __shared__ float s_inv[128];
     __shared__ float s_red[kWarps];
-    using LB = LaneBlock<FMT, HAS_GAMMA>;
+    using LB = LaneBlock<FMT, HAS_GAMMA, LN>;
+    static_assert(!LN || HAS_GAMMA, "LayerNorm takes gamma");
+    const bool has_beta = LN && a.beta != nullptr;
     constexpr int E = LB::E;
 
     const int lane = threadIdx.x & 31;
@@ -320,40 +348,57 @@ prepare_kernel(PrepArgs a) {
     if (HAS_GAMMA || FMT == 0) {
         for (int64_t row = gwarp; row < M; row += nwarps) {
             const uint16_t* xr = a.X + row * K;
-            float rinv = 1.0f;
+            float rinv = 1.0f, mu = 0.0f;
             if (HAS_GAMMA) {
-                float acc = 0.0f;
-                for (int c0 = lane; c0 < nchunk; c0 += 256) {
-                    uint4 v[8];
+                // One pass in the fixed order: lane l adds f(x) over chunks
+                // l, l+32, ... element by element, then the xor butterfly.
+                auto row_sum = [&](auto f) {
+                    float acc = 0.0f;
+                    for (int c0 = lane; c0 < nchunk; c0 += 256) {
+                        uint4 v[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+                        for (int u = 0; u < 8; ++u)
+                            if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        if (c0 + 32 * u < nchunk) {
-                            float x[8];
-                            unpack_bf16x8(v[u], x);
+                        for (int u = 0; u < 8; ++u) {
+                            if (c0 + 32 * u < nchunk) {
+                                float x[8];
+                                unpack_bf16x8(v[u], x);
 #pragma unroll
-                            for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, __fmul_rn(x[t], x[t]));
+                                for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, f(x[t]));
+                            }
                         }
                     }
-                }
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1)
-                    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
-                float ms = __fdiv_rn(acc, (float)K);
-                rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
-                if (lane == 0) rinv_ws[row] = rinv;
+                    for (int o = 16; o >= 1; o >>= 1)
+                        acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+                    return acc;
+                };
+                if (LN) {
+                    // LayerNorm: mean, then the centred squares (two passes)
+                    mu = __fdiv_rn(row_sum([](float x) { return x; }), (float)K);
+                    const float var = __fdiv_rn(row_sum([mu](float x) {
+                        const float d = __fsub_rn(x, mu);
+                        return __fmul_rn(d, d);
+                    }), (float)K);
+                    rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+                    if (lane == 0) { rinv_ws[row] = rinv; rinv_ws[M + row] = mu; }
+                } else {
+                    const float ms = __fdiv_rn(row_sum([](float x) { return __fmul_rn(x, x); }), (float)K);
+                    rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+                    if (lane == 0) rinv_ws[row] = rinv;
+                }
             }
             if (FMT == 0) {
                 if (HAS_GAMMA) {
                     for (int c0 = lane; c0 < nchunk; c0 += 128) {
-                        uint4 v[4], g[4];
+                        uint4 v[4], g[4], bt[LN ? 4 : 1];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             if (c0 + 32 * u < nchunk) {
                                 v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
                                 g[u] = ld_nc_v4(a.gamma + (int64_t)(c0 + 32 * u) * 8);
+                                if (LN && has_beta) bt[u] = ld_nc_v4(a.beta + (int64_t)(c0 + 32 * u) * 8);
                             }
                         }
 #pragma unroll
@@ -363,7 +408,16 @@ prepare_kernel(PrepArgs a) {
                                 unpack_bf16x8(v[u], y);
                                 unpack_bf16x8(g[u], gg);
 #pragma unroll
-                                for (int t = 0; t < 8; ++t) y[t] = __fmul_rn(__fmul_rn(y[t], rinv), gg[t]);
+                                for (int t = 0; t < 8; ++t) {
+                                    const float xv = LN ? __fsub_rn(y[t], mu) : y[t];
+                                    y[t] = __fmul_rn(__fmul_rn(xv, rinv), gg[t]);
+                                }
+                                if (LN && has_beta) {
+                                    float bb[8];
+                                    unpack_bf16x8(bt[u], bb);
+#pragma unroll
+                                    for (int t = 0; t < 8; ++t) y[t] = __fadd_rn(y[t], bb[t]);
+                                }
                                 amax = fmaxf(amax, amax8(y));
                             }
                         }
@@ -444,7 +498,7 @@ prepare_kernel(PrepArgs a) {
             const int64_t row = cur.row;
             const int cb = cur.cb;
             float y[E];
-            lb.y(y);
+            lb.y(y, has_beta);
             // the backbone's block max is the block max of y: the largest
             // entry of every group is always kept
             const float bm = amaxE<E>(y);
@@ -560,7 +614,7 @@ prepare_kernel(PrepArgs a) {
             const int64_t row = cur.row;
             const int cb = cur.cb;
             float y[16];
-            lb.y(y);
+            lb.y(y, has_beta);
             const float sdec = e4m3_to_f32(bs);
             float d[8];
             dequant8(bc.x, sdec, sb.gdec, d);
@@ -588,9 +642,9 @@ prepare_kernel(PrepArgs a) {
     }
 }
 
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false, bool LN = false>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
-    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS>;
+    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN>;
     static int blocks_per_sm = 0;          // same for every device of one architecture
     if (blocks_per_sm == 0) {
         int b = 0;
@@ -618,20 +672,20 @@ cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     return cudaLaunchKernelEx(&cfg, kfn, a);
 }
 
-template <int FMT, bool HAS_GAMMA, bool WEIGHT, bool RS = false>
+template <int FMT, bool HAS_GAMMA, bool WEIGHT, bool RS = false, bool LN = false>
 cudaError_t launch_m(const PrepArgs& a, int m, cudaStream_t s, int sms) {
     switch (m) {
-        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false, RS>(a, s, sms);
-        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true, RS>(a, s, sms)
-                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false, RS>(a, s, sms);
-        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false, RS>(a, s, sms);
+        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false, RS, LN>(a, s, sms);
+        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true, RS, LN>(a, s, sms)
+                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false, RS, LN>(a, s, sms);
+        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false, RS, LN>(a, s, sms);
     }
 }
 
 }  // namespace
 
 size_t prepare_ws_bytes(int64_t M) {
-    size_t b = 64 + (size_t)(M > 0 ? M : 0) * 4;
+    size_t b = 64 + (size_t)(M > 0 ? M : 0) * 8;
     return (b + 255) / 256 * 256;
 }
 
@@ -639,6 +693,7 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     PrepArgs a;
     a.X = static_cast<const uint16_t*>(p.X);
     a.gamma = static_cast<const uint16_t*>(p.gamma);
+    a.beta = static_cast<const uint16_t*>(p.beta);
     a.eps = p.eps;
     a.M = p.M;
     a.K = p.K;
@@ -657,6 +712,11 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     if (p.weight) {
         return p.fmt == 0 ? launch_one<0, false, 8, true, false>(a, s, sms)
                           : launch_one<1, false, 8, true, false>(a, s, sms);
+    }
+    if (p.layernorm) {
+        if (p.fmt == 1) return launch_m<1, true, false, false, true>(a, p.m, s, sms);
+        return p.residual_shared ? launch_m<0, true, false, true, true>(a, p.m, s, sms)
+                                 : launch_m<0, true, false, false, true>(a, p.m, s, sms);
     }
     if (p.fmt == 0 && p.residual_shared)
         return g ? launch_m<0, true, false, true>(a, p.m, s, sms) : launch_m<0, false, false, true>(a, p.m, s, sms);

@@ -13,6 +13,8 @@ namespace sharq {
 struct PrepareLaunch {
     const void* X;
     const void* gamma;
+    const void* beta;     // LayerNorm bias, may be null
+    bool layernorm;       // LayerNorm (needs gamma) instead of RMSNorm
     float eps;
     int64_t M;
     int K, n, m, fmt;

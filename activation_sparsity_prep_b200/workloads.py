@@ -98,6 +98,12 @@ def gamma_random(cfg: int, linear: int, K: int) -> np.ndarray:
     return f32_to_bf16_bits(g.astype(np.float32))
 
 
+def beta_random(cfg: int, linear: int, K: int) -> np.ndarray:
+    """A LayerNorm bias ~ N(0, 0.1) (stands in for an adaLN shift)."""
+    b = _rng(cfg, 6, linear).normal(0.0, 0.1, size=K)
+    return f32_to_bf16_bits(b.astype(np.float32))
+
+
 def routing(cfg: int, T: int, E: int, topk: int) -> np.ndarray:
     """Uniform random top-k routing: [T, topk] distinct expert ids per token."""
     g = _rng(cfg, TID_ROUTE, 0)
@@ -124,7 +130,8 @@ def group_by_expert(experts: np.ndarray, E: int) -> Tuple[np.ndarray, np.ndarray
 
 # ---------------------------------------------------------------------------
 # Workload registry: shapes follow the model families named on the pages
-# (Llama-3.1-8B, Qwen2.5-7B, Qwen3-30B-A3B); weights are random.
+# (Llama-3.1-8B, Qwen2.5-7B, Qwen3-30B-A3B, and the Wan2.2 video DiT for the
+# LayerNorm form); weights are random.
 # ---------------------------------------------------------------------------
 
 @dataclass(frozen=True)
@@ -132,8 +139,9 @@ class Linear:
     name: str
     K: int
     N: int
-    norm: bool          # fused RMSNorm on the input (gamma = 1, eps = 1e-6)
+    norm: bool          # fused norm on the input (RMSNorm: gamma = 1, eps = 1e-6)
     index: int          # linear index used in the seeds
+    layernorm: bool = False   # LayerNorm with gamma ~ U[0.5, 1.5] and beta ~ N(0, 0.1)
 
 
 @dataclass(frozen=True)
@@ -178,12 +186,26 @@ WORKLOADS: Dict[str, Workload] = {
         Ms=(16384,),
         sweep=tuple((f, n, m) for f in ("nvfp4", "mxfp4")
                     for (n, m) in ((2, 4), (1, 4), (4, 8)))),
+    # Wan2.2-T2V-A14B-shaped DiT block (hidden 5120, FFN 13824): LayerNorm
+    # (gamma = 1 + scale, beta = shift, as adaLN modulation gives) in front of
+    # the fused q/k/v and the FFN up projection; 8192 video tokens.
+    "wan_dit": Workload(
+        "wan_dit", 6, "laplace_outlier",
+        (Linear("qkv", 5120, 15360, True, 0, layernorm=True),
+         Linear("o", 5120, 5120, False, 1),
+         Linear("ffn_up", 5120, 13824, True, 2, layernorm=True),
+         Linear("ffn_down", 13824, 5120, False, 3)),
+        Ms=(8192,)),
 }
 
 
 def linear_inputs(wl: Workload, lin: Linear, M: int) -> Dict[str, np.ndarray]:
-    """X, W and gamma (or None) for one linear of a workload at M rows."""
+    """X, W, gamma (or None), beta (or None) and the norm kind ("rms" or
+    "layernorm") for one linear of a workload at M rows."""
     X = activation(wl.dist, wl.cfg, lin.index, M, lin.K, wl.n_outlier)
     W = weight(wl.cfg, lin.index, lin.N, lin.K)
+    if lin.layernorm:
+        return {"X": X, "W": W, "gamma": gamma_random(wl.cfg, lin.index, lin.K),
+                "beta": beta_random(wl.cfg, lin.index, lin.K), "norm": "layernorm"}
     g = gamma_ones(lin.K) if lin.norm else None
-    return {"X": X, "W": W, "gamma": g}
+    return {"X": X, "W": W, "gamma": g, "beta": None, "norm": "rms"}

@@ -180,7 +180,7 @@ def oracle_sample_step(linears, rows: int, quantized):
     t0 = time.perf_counter()
     fl = 0.0
     for (L, d), Wq in zip(linears, quantized):
-        P = oracle.prepare(d["X"][:rows], d["gamma"], wl.EPS)
+        P = oracle.prepare(d["X"][:rows], d["gamma"], wl.EPS, norm=d["norm"], beta=d["beta"])
         oracle.linear(P, Wq)
         fl += 2.0 * rows * L.N * L.K
     return time.perf_counter() - t0, fl
@@ -271,6 +271,7 @@ def build_units(args, dev):
         for L in W.linears:
             d = wl.linear_inputs(W, L, M)
             X, g = up(d["X"]), (None if d["gamma"] is None else up(d["gamma"]))
+            b = None if d["beta"] is None else up(d["beta"])
             Wt = up(d["W"])
             w = sq.quantize_weight(Wt, fmt)
             del Wt
@@ -278,7 +279,11 @@ def build_units(args, dev):
             ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
             Y = torch.empty((M, L.N), dtype=bf, device=dev)
             u = dict(name=L.name, rows=M, prep_rows=M, N=L.N, K=L.K, X=X, Y=Y)
-            u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
+            if L.layernorm:
+                u["prep"] = (lambda X=X, g=g, b=b, P=P, ws=ws:
+                             sq.prepare_layernorm(X, g, b, wl.EPS, n, m, fmt, out=P, ws=ws))
+            else:
+                u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
             u["gemm"] = (lambda P=P, w=w, Y=Y: sq.linear(P, w, out=Y))
             units.append(u)
         desc = (f"{W.name}: " + ", ".join(f"{L.name} {L.K}x{L.N}" for L in W.linears)

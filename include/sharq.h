@@ -118,7 +118,7 @@ SHARQ_API const char* sharq_status_string(int status);
 SHARQ_API size_t sharq_scale_bytes(int64_t rows, int K, int fmt);
 
 /* Workspace the preparation operator needs (tensor-wide maxima, a grid
- * barrier and one fp32 per row).  Caller-owned device memory; its content on
+ * barrier and two fp32 per row).  Caller-owned device memory; its content on
  * entry does not matter.  Calls that share a workspace must not overlap. */
 SHARQ_API size_t sharq_prepare_workspace_bytes(int64_t M, int K, int fmt);
 
@@ -148,6 +148,22 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_wei
 SHARQ_API sharq_status sharq_prepare(const void* X_bf16, const void* gamma_bf16, float eps,
                            const sharq_prepared* out, void* ws, size_t ws_bytes,
                            void* stream);
+
+/* The preparation operator with LayerNorm in front (the mean-subtracting
+ * norm of DiT and vision layers; the pages evaluate vision-language and
+ * video models alongside LLMs but do not define the norm's arithmetic):
+ *   mu  = sum(x) / K and var = sum((x - mu)^2) / K, each summed in the same
+ *         fixed order as the RMS sum (32 lanes, 8-element chunk c to lane
+ *         c mod 32, element order within a lane, xor butterfly 16..1);
+ *   y   = fl(fl(fl(x - mu) * rstd) * gamma) [+ beta], rstd = 1/sqrt(var+eps);
+ * then the mask, backbone and residual exactly as sharq_prepare.  gamma bf16
+ * [K] is required (SHARQ_ERR_INVALID_ARG when NULL and M > 0); beta bf16
+ * [K] may be NULL (no bias; adding a zero bias would turn -0 into +0).
+ * Same buffers, preconditions and workspace as sharq_prepare. */
+SHARQ_API sharq_status sharq_prepare_layernorm(const void* X_bf16, const void* gamma_bf16,
+                                               const void* beta_bf16, float eps,
+                                               const sharq_prepared* out, void* ws, size_t ws_bytes,
+                                               void* stream);
 
 /* Two-path FP4 linear (Abstract: a sparse FP4 GEMM on the backbone and a
  * dense FP4 GEMM on the residual, one shared weight payload):

@@ -32,7 +32,7 @@ def test_scale_and_workspace_sizes():
     assert sq.scale_bytes(129, 4096, "nvfp4") == 256 * 256
     assert sq.scale_bytes(128, 4096, "mxfp4") == 128 * 128
     assert sq.scale_bytes(16, 100, "nvfp4") == 0          # K % 256 != 0
-    assert sq.prepare_workspace_bytes(1000, 4096) >= 64 + 4 * 1000
+    assert sq.prepare_workspace_bytes(1000, 4096) >= 64 + 8 * 1000
     assert sq.scale_bytes(0, 256) == 0
 
 
@@ -100,3 +100,20 @@ def test_unknown_residual_scale_is_rejected_everywhere():
     assert L.sharq_moe_linear(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000, 0,
                               0x1000, ws, None) == 1
     assert L.sharq_prepare_noalloc(0x1000, None, 1e-6, ctypes.byref(cp), None) == 1
+
+
+def test_layernorm_prepare_needs_gamma_and_aligned_beta():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    assert L.sharq_prepare_layernorm(0x1000, None, None, 1e-6, ctypes.byref(cp), 0x1000, 1 << 20, None) == 1
+    assert L.sharq_prepare_layernorm(0x1000, 0x1000, 0x1004, 1e-6, ctypes.byref(cp), 0x1000, 1 << 20, None) == 1
+    assert sq.prepare_workspace_bytes(1000, 4096) >= 64 + 8 * 1000      # mean and rstd per row
+
+
+def test_workload_inputs_carry_the_norm_kind():
+    from activation_sparsity_prep_b200 import workloads as wl
+    W = wl.WORKLOADS["wan_dit"]
+    d = wl.linear_inputs(W, W.linears[0], 4)
+    assert d["norm"] == "layernorm" and d["beta"].shape == (5120,) and d["gamma"].shape == (5120,)
+    d = wl.linear_inputs(W, W.linears[1], 4)
+    assert d["norm"] == "rms" and d["gamma"] is None and d["beta"] is None

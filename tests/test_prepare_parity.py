@@ -92,6 +92,49 @@ def test_prepare_shared_residual_scale_bit_exact(M, K, dist, gk, n, m):
     assert torch.equal(P.rs_tscale, P.bb_tscale)
 
 
+LN_CASES = [
+    # M, K, dist, beta, n, m, fmt, residual
+    (16, 256, "normal_outlier", True, 2, 4, "nvfp4", "own"),
+    (3, 768, "laplace_outlier", False, 2, 4, "nvfp4", "own"),
+    (129, 5120, "laplace_outlier", True, 2, 4, "nvfp4", "own"),
+    (300, 1024, "student_t", True, 1, 4, "nvfp4", "shared"),
+    (64, 2048, "laplace_outlier", True, 4, 8, "mxfp4", "own"),
+    (600, 4096, "student_t", False, 2, 4, "mxfp4", "own"),
+]
+
+
+@pytest.mark.parametrize("M,K,dist,hb,n,m,fmt,rs", LN_CASES)
+def test_prepare_layernorm_bit_exact(M, K, dist, hb, n, m, fmt, rs):
+    X = wl.activation(dist, 25, M + K, M, K)
+    g = wl.gamma_random(25, 0, K)
+    b = wl.beta_random(25, 0, K) if hb else None
+    P = sq.prepare_layernorm(to_dev(X), to_dev(g), None if b is None else to_dev(b), 1e-6, n, m, fmt,
+                             want_mask=True, residual_scale=rs)
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    R = oracle.prepare(X, g, 1e-6, n, m, fmt, residual_scale=rs, norm="layernorm", beta=b)
+    assert np.array_equal(to_np(P.mask), R.mask), "mask"
+    assert np.array_equal(to_np(P.bb_codes), R.bb.codes), "backbone codes"
+    assert np.array_equal(to_np(P.rs_codes), R.rs.codes), "residual codes"
+    assert np.array_equal(atoms_to_canonical(to_np(P.bb_scales), M, K, fmt), R.bb.scales)
+    assert np.array_equal(atoms_to_canonical(to_np(P.rs_scales), M, K, fmt), R.rs.scales)
+    assert to_np(P.bb_tscale).view(np.uint32)[0] == np.float32(R.bb.tscale).view(np.uint32)
+    assert to_np(P.rs_tscale).view(np.uint32)[0] == np.float32(R.rs.tscale).view(np.uint32)
+
+
+def test_prepare_layernorm_constant_rows_give_beta():
+    """Constant rows normalise to exactly beta: the backbone and residual
+    are those of the tensor [beta; beta; ...] with no norm."""
+    K = 512
+    b = wl.beta_random(26, 0, K)
+    X = np.repeat(wl.f32_to_bf16_bits(np.full((1, K), 2.5, np.float32)), 8, axis=0)
+    P = sq.prepare_layernorm(to_dev(X), to_dev(wl.gamma_random(26, 0, K)), to_dev(b))
+    Q = sq.prepare(to_dev(np.repeat(b[None], 8, axis=0)), None)
+    torch.cuda.synchronize()
+    assert torch.equal(P.bb_codes, Q.bb_codes) and torch.equal(P.rs_codes, Q.rs_codes)
+    assert torch.equal(P.bb_scales, Q.bb_scales) and torch.equal(P.rs_tscale, Q.rs_tscale)
+
+
 def test_prepare_special_values():
     """Rows of zeros, -0, exact ties inside groups, a constant row, values at
     E2M1/E4M3 rounding boundaries and one huge outlier."""
