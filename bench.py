@@ -45,7 +45,7 @@ PREP_BYTES_PER_ELEM = {(0, 1): 3.125, (1, 1): 3.0625}   # (fmt, zero-filled back
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
     ap.add_argument("--workload", default="llama8b")
@@ -75,11 +75,31 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+# --------------------------------------------------------- multi-rank ----
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The slowest rank's figure (every rank returns it); identity on one
+    rank.  The tensor lives on `device` (cuda for NCCL, cpu for gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_step: float, world: int, steps: int, total_ms: float) -> float:
+    """Weak scaling: every rank does `work_per_step` per step, the job takes
+    the slowest rank's time."""
+    return work_per_step * world * steps / (total_ms * 1e-3)
+
+
 # ------------------------------------------------------------- clocks ----
 
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons while running."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -87,6 +107,10 @@ class ClockSampler:
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.window = None       # (start, end) of the timed region, host epoch seconds
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -94,7 +118,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "10"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -113,26 +137,34 @@ class ClockSampler:
     def summary(self):
         if not self.path or not os.path.exists(self.path):
             return None
-        sm, smax, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
+                ts = parts[0]
+                t = time.mktime(time.strptime(ts.split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                t += float("0." + ts.split(".")[1]) if "." in ts else 0.0
+                rows.append((t, float(parts[2]), float(parts[3]),
+                             {n for n, v in zip(names, parts[6:10]) if v.lower() == "active"}))
+            except (ValueError, IndexError):
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
         os.unlink(self.path)
-        if not sm:
+        if not rows:
             return None
-        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = rows
+        where = "all samples (none fell inside the timed region)"
+        if self.window:
+            w = [r for r in rows if self.window[0] - 0.005 <= r[0] <= self.window[1] + 0.005]
+            if w:
+                inside, where = w, "samples inside the timed region"
+        sm = [r[1] for r in inside]
+        reasons = set().union(*[r[3] for r in inside])
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": sorted(reasons), "samples": len(inside), "window": where,
+                "interval_ms": 10}
 
 
 # ------------------------------------------------------------- inputs ----
@@ -173,17 +205,59 @@ def profiled_traffic(launch_key: str, sha: str):
 
 # ------------------------------------------------------------ CPU arm ----
 
-def oracle_sample_step(linears, rows: int, quantized):
+def oracle_sample_step(linears, rows: int, quantized, fmt="nvfp4", n=2, m=4, residual="own"):
     """One bounded oracle step: prepare and linear of the first `rows` rows
     of every linear.  Returns (seconds, effective flops of the sample)."""
     import oracle
     t0 = time.perf_counter()
     fl = 0.0
     for (L, d), Wq in zip(linears, quantized):
-        P = oracle.prepare(d["X"][:rows], d["gamma"], wl.EPS, norm=d["norm"], beta=d["beta"])
+        P = oracle.prepare(d["X"][:rows], d["gamma"], wl.EPS, n, m, fmt, residual_scale=residual,
+                           norm=d["norm"], beta=d["beta"])
         oracle.linear(P, Wq)
         fl += 2.0 * rows * L.N * L.K
     return time.perf_counter() - t0, fl
+
+
+def oracle_moe_sample_step(W, sample, fmt="nvfp4", n=2, m=4, residual="own"):
+    """Bounded oracle step of the grouped layer: every sampled dispatched row
+    through its own expert's two-path linear."""
+    import oracle
+    t0 = time.perf_counter()
+    fl = 0.0
+    for li, (L, X, g, rows, experts, wq) in enumerate(sample):
+        P = oracle.prepare(X, g, wl.EPS, n, m, fmt, residual_scale=residual)
+        for e in sorted(set(experts.tolist())):
+            sel = np.nonzero(experts == e)[0].astype(np.int32)
+            oracle.linear(oracle.gather_rows(P, rows[sel]), wq[e])
+            fl += 2.0 * len(sel) * L.N * L.K
+    return time.perf_counter() - t0, fl
+
+
+def moe_reference_sample(W, fmt, tokens: int = 4):
+    """Sampled operands of the grouped layer: the first `tokens` tokens for
+    gate+up (each with its top-k experts) and the first tokens*top-k
+    dispatched rows for down, with only the experts they reach quantised."""
+    import oracle
+    T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
+    ex = wl.routing(W.cfg, T, E, topk)
+    ri, off = wl.group_by_expert(ex.astype(np.int32), E)
+    sample = []
+    for li, L in enumerate(W.linears):
+        if li == 0:
+            X = wl.activation(W.dist, W.cfg, L.index, tokens, L.K)
+            rows = np.repeat(np.arange(tokens, dtype=np.int32), topk)
+            experts = ex[:tokens].reshape(-1)
+        else:
+            nrow = tokens * topk
+            X = wl.activation(W.dist, W.cfg, L.index, T * topk, L.K)[:nrow]
+            rows = np.arange(nrow, dtype=np.int32)
+            experts = (np.searchsorted(off, rows, side="right") - 1).astype(np.int64)
+        g = wl.gamma_ones(L.K) if L.norm else None
+        wq = {int(e): oracle.quantize_weight(wl.weight(W.cfg * 1000 + li, 100 + int(e), L.N, L.K), fmt)
+              for e in set(experts.tolist())}
+        sample.append((L, X, g, rows, experts, wq))
+    return sample
 
 
 def blas_threads():
@@ -195,20 +269,39 @@ def blas_threads():
         return 1
 
 
-def cpu_baseline(linears, budget_s: float = 15.0, rows: int = 16):
+def cpu_baseline(linears, args, budget_s: float = 15.0, rows: int = 16):
     import oracle
-    quantized = [oracle.quantize_weight(d["W"]) for _, d in linears]
+    n_, m_ = nm_of(args)
+    quantized = [oracle.quantize_weight(d["W"], args.fmt) for _, d in linears]
     total_t, total_f, n = 0.0, 0.0, 0
     while total_t < budget_s and n < 50:
-        t, f = oracle_sample_step(linears, rows, quantized)
+        t, f = oracle_sample_step(linears, rows, quantized, args.fmt, n_, m_, args.residual)
         total_t += t
         total_f += f
         n += 1
     return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
             "kind": "oracle",
             "sample": f"{n} passes of: oracle prepare + fp64 two-path linear on the first {rows} "
-                      f"rows of each of the 4 linears (all N); prepare single-threaded C, "
+                      f"rows of each of the {len(linears)} linears (all N); prepare single-threaded C, "
                       f"GEMM numpy/OpenBLAS fp64"}
+
+
+def workload_desc(W, M):
+    """The workload description both arms put in config["workload"]."""
+    if W.moe is None:
+        return (f"{W.name}: " + ", ".join(f"{L.name} {L.K}x{L.N}" for L in W.linears)
+                + f"; M={M}, prepare+linear each")
+    T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
+    return (f"{W.name}: Qwen3-30B-A3B-shaped expert layer, {T} tokens, {E} experts, top-{topk}; "
+            f"gate_up {W.linears[0].K}x{W.linears[0].N} (rows gathered by index), "
+            f"down {W.linears[1].K}x{W.linears[1].N} (rows in dispatch order); grouped prepare+linear")
+
+
+def bench_config(args, W, M):
+    return {"workload": workload_desc(W, M), "M": M, "fmt": args.fmt, "nm": args.nm,
+            "residual_scale": args.residual,
+            "l2": "flushed between timed steps (512 MiB write)",
+            "timing": "CUDA graph per step, per-kernel external events"}
 
 
 def run_reference(args):
@@ -216,30 +309,40 @@ def run_reference(args):
     if rank != 0:
         return 0
     W = wl.WORKLOADS[args.workload]
-    linears = make_inputs(W, args.M)
-    import oracle
-    quantized = [oracle.quantize_weight(d["W"]) for _, d in linears]
-    rows = 16
+    n, m = nm_of(args)
+    cores = blas_threads()
+    if W.moe is None:
+        linears = make_inputs(W, args.M)
+        import oracle
+        quantized = [oracle.quantize_weight(d["W"], args.fmt) for _, d in linears]
+        rows = 16
+        step = lambda: oracle_sample_step(linears, rows, quantized, args.fmt, n, m, args.residual)
+        what = f"first {rows} rows of each linear per step (all N), of M={args.M}"
+        M = args.M
+    else:
+        sample = moe_reference_sample(W, args.fmt)
+        step = lambda: oracle_moe_sample_step(W, sample, args.fmt, n, m, args.residual)
+        what = ("4 tokens through gate+up (each with its top-8 experts) and the first 32 dispatched "
+                "rows through down, per step")
+        M = W.moe["T"]
     for _ in range(args.warmup):
-        oracle_sample_step(linears, rows, quantized)
+        step()
     times, fl = [], 0.0
     for _ in range(args.steps):
-        t, f = oracle_sample_step(linears, rows, quantized)
+        t, f = step()
         times.append(t)
         fl = f
     tot = sum(times)
     value = fl * args.steps / tot / 1e12
-    cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 GEMM over FP4-decoded operands; f32 prepare",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload} decoder linears, sample of {rows} rows per linear "
-                               f"(of M={args.M})", "M_sampled": rows, "fmt": "nvfp4", "nm": "2:4"},
+        "config": bench_config(args, W, M),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"first {rows} rows of each linear per step"},
+                         "sample": what + "; prepare single-threaded C, GEMM numpy/OpenBLAS fp64"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -286,9 +389,7 @@ def build_units(args, dev):
                 u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
             u["gemm"] = (lambda P=P, w=w, Y=Y: sq.linear(P, w, out=Y))
             units.append(u)
-        desc = (f"{W.name}: " + ", ".join(f"{L.name} {L.K}x{L.N}" for L in W.linears)
-                + f"; M={M}, prepare+linear each")
-        return units, desc, M
+        return units, M
     T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
     ri, off = wl.group_by_expert(wl.routing(W.cfg, T, E, topk), E)
     ri_d = torch.from_numpy(ri).to(dev)
@@ -313,10 +414,7 @@ def build_units(args, dev):
         u["gemm"] = (lambda P=P, w=w, Y=Y, rix=rix, mws=mws:
                      sq.moe_linear(P, rix, off_d, w, out=Y, ws=mws, T=T * topk))
         units.append(u)
-    desc = (f"{W.name}: Qwen3-30B-A3B-shaped expert layer, {T} tokens, {E} experts, top-{topk}; "
-            f"gate_up {W.linears[0].K}x{W.linears[0].N} (rows gathered by index), "
-            f"down {W.linears[1].K}x{W.linears[1].N} (rows in dispatch order); grouped prepare+linear")
-    return units, desc, T
+    return units, T
 
 
 def run_sharq(args):
@@ -333,7 +431,7 @@ def run_sharq(args):
     dev = torch.device("cuda", local)
     fmt = sq._FMT[args.fmt]
     n, m = nm_of(args)
-    units, desc, tokens_per_step = build_units(args, dev)
+    units, tokens_per_step = build_units(args, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def step():
@@ -369,6 +467,7 @@ def run_sharq(args):
     torch.cuda.synchronize()
     step_ms, prep_ms, lin_ms = [], [[] for _ in units], [[] for _ in units]
     with ClockSampler(local) as clk:
+        t_start = time.time()
         for _ in range(args.steps):
             flush.zero_()                    # L2 flushed between timed steps
             g.replay()
@@ -377,20 +476,18 @@ def run_sharq(args):
             for i in range(len(units)):
                 prep_ms[i].append(evs[2 * i].elapsed_time(evs[2 * i + 1]))
                 lin_ms[i].append(evs[2 * i + 1].elapsed_time(evs[2 * i + 2]))
+        clk.mark(t_start, time.time())
     torch.cuda.synchronize()
     status = sq.last_device_status()
-    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), dev)
     if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
     clocks = clk.summary()
 
     fl_step = sum(2.0 * u["rows"] * u["N"] * u["K"] for u in units)
     ms_step = total_ms / args.steps
-    value = fl_step * world * args.steps / (total_ms * 1e-3) / 1e12
-    tokens = tokens_per_step * world * args.steps / (total_ms * 1e-3)
+    value = whole_job_rate(fl_step, world, args.steps, total_ms) / 1e12
+    tokens = whole_job_rate(tokens_per_step, world, args.steps, total_ms)
 
     hbm, bf16, src = peaks()
     fp4_peak = 4.0 * bf16           # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PFLOP/s)
@@ -444,20 +541,17 @@ def run_sharq(args):
             torch.cuda.synchronize()
             if it >= args.warmup:
                 ts.append(e0.elapsed_time(e1))
-        tot = sum(ts)
-        if world > 1:
-            t = torch.tensor([tot], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            tot = float(t.item())
-        e2e = {"value": fl_step * world * args.steps / (tot * 1e-3) / 1e12, "unit": "TFLOP/s",
+        tot = max_over_ranks(sum(ts), dev)
+        e2e = {"value": whole_job_rate(fl_step, world, args.steps, tot) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hx)),
                "d2h_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hy)),
                "ms_per_step": tot / args.steps}
 
     base = None
-    if (rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "llama8b"):
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline
+            and wl.WORKLOADS[args.workload].moe is None):
         linears = make_inputs(wl.WORKLOADS[args.workload], args.M)
-        base = cpu_baseline(linears)
+        base = cpu_baseline(linears, args)
 
     if rank == 0:
         line = {
@@ -465,10 +559,7 @@ def run_sharq(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4" if fmt == 0 else "mxfp4", "data": "synthetic",
-            "config": {"workload": desc, "M": tokens_per_step, "fmt": args.fmt, "nm": args.nm,
-                       "residual_scale": args.residual,
-                       "l2": "flushed between timed steps (512 MiB write)",
-                       "timing": "CUDA graph per step, per-kernel external events"},
+            "config": bench_config(args, wl.WORKLOADS[args.workload], tokens_per_step),
             "tokens_per_s": tokens,
             "roofline": {"bound": "hbm" if hbm_bound else "tensor", "achieved": achieved,
                          "peak": lin_peak, "unit": lin_unit, "frac": achieved / lin_peak,
