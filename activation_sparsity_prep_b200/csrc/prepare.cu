@@ -55,11 +55,6 @@ __device__ __forceinline__ float* ws_rinv(uint32_t* ws) {
     return reinterpret_cast<float*>(ws + 16);
 }
 
-// LayerNorm means follow the M per-row reciprocals.
-__device__ __forceinline__ float* ws_mu(uint32_t* ws, int64_t M) {
-    return reinterpret_cast<float*>(ws + 16) + M;
-}
-
 // Byte offset of scale (row, s) in the MMA-ready atom layout.
 __device__ __forceinline__ int64_t sf_off(int64_t row, int s, int nsf) {
     return ((row >> 7) * (int64_t)(nsf >> 2) + (s >> 2)) * 512 + (row & 31) * 16 +
@@ -281,7 +276,7 @@ struct LaneBlock {
             rinv = rinv_ws[row];
         }
         if (LN) {
-            mu = rinv_ws[a.M + row];
+            mu = rinv_ws[a.M + row];          // the LayerNorm means follow the M reciprocals
             if (a.beta) {
 #pragma unroll
                 for (int v = 0; v < NV; ++v) b[v] = ld_nc_v4(a.beta + (int64_t)cb * E + 8 * v);
