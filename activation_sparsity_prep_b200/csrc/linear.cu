@@ -452,6 +452,215 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, kTmemCols); }
 }
 
+// ------------------------------------------------------------------------
+// Decode form (M <= 64 rows).  With few rows a 128-row activation tile is
+// almost all padding and a 128 x 128 MMA spends most of its work on it.
+// Here the operands swap roles: the weight tile (128 output columns) is the
+// MMA's M side and the NT activation rows its N side, so every MMA does
+// 128 x NT x 64 of useful work and the kernel streams the weight.  Both
+// paths still share each weight tile (two MMAs, A = W, B = backbone or
+// residual; the activation scale atoms serve as the B-side scales, whose
+// first NT rows the MMA reads).  The accumulators hold Y^T; the epilogue
+// writes them transposed.  Warp roles as in linear_kernel.
+// ------------------------------------------------------------------------
+template <int FMT, int NT>
+struct DecCfg {
+    using C = Cfg<FMT>;
+    static constexpr uint32_t kActBytes = NT * (BK / 2);          // one activation tile
+    static constexpr uint32_t kStageBytes = kTileBytes + 2 * kActBytes + 3 * C::kSfBytes;
+    static constexpr uint32_t kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+    static constexpr int kStagesRaw = (200 * 1024) / (int)kStageStride;
+    static constexpr int S = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr uint32_t kSfCols = 3 * 4 * C::kAtoms;         // per stage
+    static constexpr uint32_t kAccCols = 4 * NT;                   // two buffers x two paths
+    static_assert(kAccCols + S * kSfCols <= kTmemCols, "tensor memory budget");
+    // E2M1 A and B, K-major, N = NT, M = 128 (see Cfg::kIdesc)
+    static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) |
+                                       ((uint32_t)FMT << 23) | ((uint32_t)(BM >> 4) << 24);
+};
+
+template <int S>
+struct alignas(8) DecBarriers {
+    uint64_t full[S];
+    uint64_t empty[S];        // MMAs done + scale warps done reading
+    uint64_t sf_full[S];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint32_t tmem_base;
+};
+
+template <int FMT>
+__device__ __forceinline__ void mma_id(uint32_t idesc0, uint32_t d, uint64_t a, uint64_t b,
+                                       uint32_t sfa, uint32_t sfb, uint32_t acc, uint32_t sf_id) {
+    const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
+    const uint32_t hi = sf_id << 30;
+    if (FMT == 0) tc_mma_nvf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
+    else          tc_mma_mxf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
+}
+
+template <int FMT, bool ONE, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
+              const __grid_constant__ CUtensorMap tm_r, const uint8_t* __restrict__ sf_w,
+              const uint8_t* __restrict__ sf_b, const uint8_t* __restrict__ sf_r, int K,
+              EpiArgs ep, int ntiles) {
+    using C = Cfg<FMT>;
+    using D = DecCfg<FMT, NT>;
+    constexpr int S = D::S;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    DecBarriers<S>* bars = reinterpret_cast<DecBarriers<S>*>(smem + S * D::kStageStride);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nk = K / BK;
+    const int nsf = K / C::BS;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1 + 4);
+            mbar_init(&bars->sf_full[s], 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->acc_full[b], 1);
+            mbar_init(&bars->acc_empty[b], 4);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) { tmem_alloc(&bars->tmem_base, kTmemCols); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t t_sf0 = tmem + D::kAccCols;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_w); prefetch_tmap(&tm_b); prefetch_tmap(&tm_r);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const uint8_t* gw = sf_w + (int64_t)tile * (nsf / 4) * 512;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t s = it % S;
+                    if (it >= (uint32_t)S && !mbar_wait(&bars->empty[s], ((it / S) - 1) & 1)) { ok = false; break; }
+                    uint8_t* st = smem + s * D::kStageStride;
+                    mbar_arrive_expect_tx(&bars->full[s], D::kStageBytes);
+                    tma_load_2d(st, &tm_w, &bars->full[s], kb * (BK / 2), tile * BM);
+                    tma_load_2d(st + kTileBytes, &tm_b, &bars->full[s], kb * (BK / 2), 0);
+                    tma_load_2d(st + kTileBytes + D::kActBytes, &tm_r, &bars->full[s], kb * (BK / 2), 0);
+                    const int64_t sfo = (int64_t)kb * C::kAtoms * 512;
+                    uint8_t* sfs = st + kTileBytes + 2 * D::kActBytes;
+                    bulk_load(sfs, gw + sfo, C::kSfBytes, &bars->full[s]);
+                    bulk_load(sfs + C::kSfBytes, sf_b + sfo, C::kSfBytes, &bars->full[s]);
+                    bulk_load(sfs + 2 * C::kSfBytes, sf_r + sfo, C::kSfBytes, &bars->full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+                const uint32_t buf = tc & 1u, use = tc >> 1;
+                if (use > 0 && !mbar_wait(&bars->acc_empty[buf], (use - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_b = tmem + buf * 2 * NT;
+                const uint32_t d_r = ONE ? d_b : d_b + NT;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t s = it % S;
+                    if (!mbar_wait(&bars->full[s], (it / S) & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars->sf_full[s], (it / S) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    uint8_t* st = smem + s * D::kStageStride;
+                    const uint32_t a_w = smem_u32(st), a_b = smem_u32(st + kTileBytes);
+                    const uint32_t a_r = smem_u32(st + kTileBytes + D::kActBytes);
+                    const uint32_t t_sfw = t_sf0 + s * D::kSfCols;
+                    const uint32_t t_sfb = t_sfw + 4 * C::kAtoms, t_sfr = t_sfb + 4 * C::kAtoms;
+#pragma unroll
+                    for (int j = 0; j < BK / 64; ++j) {
+                        const int at = j / C::kStepsPerAtom;
+                        const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
+                        const uint32_t col = 4 * at;
+                        const uint64_t dw = sdesc_sw128(a_w + 32 * j);
+                        const uint32_t acc = (kb | j) ? 1u : 0u;
+                        mma_id<FMT>(D::kIdesc, d_b, dw, sdesc_sw128(a_b + 32 * j), t_sfw + col, t_sfb + col,
+                                    acc, sf_id);
+                        mma_id<FMT>(D::kIdesc, d_r, dw, sdesc_sw128(a_r + 32 * j), t_sfw + col, t_sfr + col,
+                                    ONE ? 1u : acc, sf_id);
+                    }
+                    tc_commit(&bars->empty[s]);
+                }
+                tc_commit(&bars->acc_full[buf]);
+            }
+        }
+    } else if (warp >= 6) {
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const uint32_t s = it % S;
+                if (!mbar_wait(&bars->full[s], (it / S) & 1)) { ok = false; break; }
+                const uint8_t* sf = smem + s * D::kStageStride + kTileBytes + 2 * D::kActBytes;
+                const uint32_t tcol = t_sf0 + s * D::kSfCols + lane_off;
+#pragma unroll
+                for (int o = 0; o < 3; ++o) {
+                    uint4 v[C::kAtoms];
+#pragma unroll
+                    for (int at = 0; at < C::kAtoms; ++at)
+                        v[at] = ld_shared_v4(sf + o * C::kSfBytes + 512 * at + 16 * lane);
+                    if constexpr (C::kAtoms == 4) tmem_st_32x32b_x16(tcol + o * 4 * C::kAtoms, v);
+                    else                          tmem_st_32x32b_x8(tcol + o * 4 * C::kAtoms, v);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) { mbar_arrive(&bars->sf_full[s]); mbar_arrive(&bars->empty[s]); }
+            }
+        }
+    } else {
+        // Epilogue: warp w reads TMEM lanes 32*(w%4).. = output columns of the
+        // tile; each thread holds its column's NT rows.
+        const int q = warp & 3;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const float gwv = ep.w_tscale[0];
+        const float gb = *ep.bb_tscale * gwv, gr = *ep.rs_tscale * gwv;
+        const int rows = (int)(ep.M < NT ? ep.M : NT);
+        uint32_t tc = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+            const uint32_t buf = tc & 1u, use = tc >> 1;
+            const bool ok = mbar_wait(&bars->acc_full[buf], use & 1);
+            tc_fence_after();
+            if (!ok) break;
+            const uint32_t src_b = tmem + buf * 2 * NT + lane_off;
+            const int64_t col = (int64_t)tile * BM + q * 32 + lane;
+#pragma unroll
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                uint32_t vb[16], vr[16];
+                tmem_ld_32x32b_x16(src_b + c0, vb);
+                if (!ONE) tmem_ld_32x32b_x16(src_b + NT + c0, vr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    if (c0 + t < rows) {
+                        const float y = ONE ? gb * __uint_as_float(vb[t])
+                                            : gb * __uint_as_float(vb[t]) + gr * __uint_as_float(vr[t]);
+                        const int64_t idx = (int64_t)(c0 + t) * ep.N + col;
+                        if (ep.y_fp32) static_cast<float*>(ep.Y)[idx] = y;
+                        else           static_cast<__nv_bfloat16*>(ep.Y)[idx] = __float2bfloat16_rn(y);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, kTmemCols); }
+}
+
 // ------------------------------------------------------------------ host --
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -535,8 +744,44 @@ cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void*
                                                 W_rows, sc, max_tiles, s, sms);
 }
 
+template <int FMT, bool ONE, int NT>
+cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
+    using D = DecCfg<FMT, NT>;
+    CUtensorMap tb, tr, tw;
+    if (!make_code_map(&tw, p.w_codes, p.N, p.K / 2, BM) ||
+        !make_code_map(&tb, p.bb_codes, p.M, p.K / 2, NT) ||
+        !make_code_map(&tr, p.rs_codes, p.M, p.K / 2, NT))
+        return cudaErrorInvalidValue;
+    const size_t smem = D::S * D::kStageStride + sizeof(DecBarriers<D::S>) + 1024;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<FMT, ONE, NT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
+    const int ntiles = p.N / BN;
+    const int grid = std::max(1, std::min(ntiles, std::max(1, sms)));
+    decode_kernel<FMT, ONE, NT><<<grid, kThreads, smem, s>>>(
+        tw, tb, tr, static_cast<const uint8_t*>(p.w_scales), static_cast<const uint8_t*>(p.bb_scales),
+        static_cast<const uint8_t*>(p.rs_scales), p.K, ep, ntiles);
+    return cudaGetLastError();
+}
+
+template <int FMT, int NT>
+cudaError_t launch_decode_nt(const LinearLaunch& p, cudaStream_t s, int sms) {
+    return p.one_acc ? launch_decode_t<FMT, true, NT>(p, s, sms) : launch_decode_t<FMT, false, NT>(p, s, sms);
+}
+
 template <int FMT>
 cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
+    // few rows: the swapped (weight-streaming) form
+    if (p.M <= 16) return launch_decode_nt<FMT, 16>(p, s, sms);
+    if (p.M <= 32) return launch_decode_nt<FMT, 32>(p, s, sms);
+    if (p.M <= 64) return launch_decode_nt<FMT, 64>(p, s, sms);
     Sched sc{};
     sc.mt_count = (int)((p.M + BM - 1) / BM);
     sc.nt_count = p.N / BN;

@@ -94,6 +94,11 @@ SHAPES = [
     (128, 128, 2048, "nvfp4"),
     (16, 256, 256, "mxfp4"),
     (129, 384, 1024, "mxfp4"),
+    # few rows: the swapped (weight-streaming) form, token tiles of 16 / 32 / 64
+    (20, 384, 1024, "nvfp4"),
+    (64, 256, 2048, "nvfp4"),
+    (40, 128, 512, "mxfp4"),
+    (1, 1024, 4096, "mxfp4"),
 ]
 
 
