@@ -161,6 +161,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// ----------------------------------------------------------- clusters ----
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Hardware barrier of every thread of every CTA in the cluster (release /
+// acquire on shared::cluster).  Every thread of the cluster must reach it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// fp32 at a shared-memory address of CTA `rank` of this cluster.
+__device__ __forceinline__ float ld_shared_cluster_f32(const void* local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r) : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------- TMA -------
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar,

@@ -462,6 +462,11 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
 // residual; the activation scale atoms serve as the B-side scales, whose
 // first NT rows the MMA reads).  The accumulators hold Y^T; the epilogue
 // writes them transposed.  Warp roles as in linear_kernel.
+// When there are fewer output tiles than SMs, a cluster of `split` CTAs
+// shares each tile, CTA rank r taking the r-th contiguous range of K
+// steps; each drains its partial (already scaled by the tensor scales)
+// into its shared memory and rank 0 sums the partials in rank order over
+// distributed shared memory before storing Y.
 // ------------------------------------------------------------------------
 template <int FMT, int NT>
 struct DecCfg {
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_r, const uint8_t* __restrict__ sf_w,
               const uint8_t* __restrict__ sf_b, const uint8_t* __restrict__ sf_r, int K,
-              EpiArgs ep, int ntiles) {
+              EpiArgs ep, int ntiles, int split) {
     using C = Cfg<FMT>;
     using D = DecCfg<FMT, NT>;
     constexpr int S = D::S;
@@ -532,15 +537,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const uint32_t t_sf0 = tmem + D::kAccCols;
+    // split > 1: one tile per cluster, this CTA's range of k-steps
+    const int krank = split > 1 ? (int)cluster_ctarank() : 0;
+    const int k0 = nk * krank / split, k1 = nk * (krank + 1) / split;
+    const int tile0 = blockIdx.x / split, tstride = gridDim.x / split;
+    float* partial = reinterpret_cast<float*>(smem);           // [NT][BM], stage memory reused
 
     if (warp == 0) {
         if (lane == 0) {
             prefetch_tmap(&tm_w); prefetch_tmap(&tm_b); prefetch_tmap(&tm_r);
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            for (int tile = tile0; tile < ntiles && ok; tile += tstride) {
                 const uint8_t* gw = sf_w + (int64_t)tile * (nsf / 4) * 512;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                for (int kb = k0; kb < k1; ++kb, ++it) {
                     const uint32_t s = it % S;
                     if (it >= (uint32_t)S && !mbar_wait(&bars->empty[s], ((it / S) - 1) & 1)) { ok = false; break; }
                     uint8_t* st = smem + s * D::kStageStride;
@@ -560,13 +570,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         if (lane == 0) {
             uint32_t it = 0, tc = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+            for (int tile = tile0; tile < ntiles && ok; tile += tstride, ++tc) {
                 const uint32_t buf = tc & 1u, use = tc >> 1;
                 if (use > 0 && !mbar_wait(&bars->acc_empty[buf], (use - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_b = tmem + buf * 2 * NT;
                 const uint32_t d_r = ONE ? d_b : d_b + NT;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                for (int kb = k0; kb < k1; ++kb, ++it) {
                     const uint32_t s = it % S;
                     if (!mbar_wait(&bars->full[s], (it / S) & 1)) { ok = false; break; }
                     if (!mbar_wait(&bars->sf_full[s], (it / S) & 1)) { ok = false; break; }
@@ -582,7 +592,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
                         const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
                         const uint32_t col = 4 * at;
                         const uint64_t dw = sdesc_sw128(a_w + 32 * j);
-                        const uint32_t acc = (kb | j) ? 1u : 0u;
+                        const uint32_t acc = (kb > k0 || j) ? 1u : 0u;
                         mma_id<FMT>(D::kIdesc, d_b, dw, sdesc_sw128(a_b + 32 * j), t_sfw + col, t_sfb + col,
                                     acc, sf_id);
                         mma_id<FMT>(D::kIdesc, d_r, dw, sdesc_sw128(a_r + 32 * j), t_sfw + col, t_sfr + col,
@@ -597,8 +607,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         uint32_t it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-            for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int tile = tile0; tile < ntiles && ok; tile += tstride) {
+            for (int kb = k0; kb < k1; ++kb, ++it) {
                 const uint32_t s = it % S;
                 if (!mbar_wait(&bars->full[s], (it / S) & 1)) { ok = false; break; }
                 const uint8_t* sf = smem + s * D::kStageStride + kTileBytes + 2 * D::kActBytes;
@@ -627,13 +637,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         const float gb = *ep.bb_tscale * gwv, gr = *ep.rs_tscale * gwv;
         const int rows = (int)(ep.M < NT ? ep.M : NT);
         uint32_t tc = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+        for (int tile = tile0; tile < ntiles; tile += tstride, ++tc) {
             const uint32_t buf = tc & 1u, use = tc >> 1;
             const bool ok = mbar_wait(&bars->acc_full[buf], use & 1);
             tc_fence_after();
             if (!ok) break;
             const uint32_t src_b = tmem + buf * 2 * NT + lane_off;
             const int64_t col = (int64_t)tile * BM + q * 32 + lane;
+            const int jl = q * 32 + lane;                     // column within the tile
 #pragma unroll
             for (int c0 = 0; c0 < NT; c0 += 16) {
                 uint32_t vb[16], vr[16];
@@ -645,9 +656,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
                     if (c0 + t < rows) {
                         const float y = ONE ? gb * __uint_as_float(vb[t])
                                             : gb * __uint_as_float(vb[t]) + gr * __uint_as_float(vr[t]);
-                        const int64_t idx = (int64_t)(c0 + t) * ep.N + col;
-                        if (ep.y_fp32) static_cast<float*>(ep.Y)[idx] = y;
-                        else           static_cast<__nv_bfloat16*>(ep.Y)[idx] = __float2bfloat16_rn(y);
+                        if (split > 1) {
+                            partial[(c0 + t) * BM + jl] = y;
+                        } else {
+                            const int64_t idx = (int64_t)(c0 + t) * ep.N + col;
+                            if (ep.y_fp32) static_cast<float*>(ep.Y)[idx] = y;
+                            else           static_cast<__nv_bfloat16*>(ep.Y)[idx] = __float2bfloat16_rn(y);
+                        }
                     }
                 }
             }
@@ -655,6 +670,37 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
         }
+    }
+    if (split > 1) {
+        // every CTA's partial is in its shared memory; rank 0 adds them in
+        // rank order and stores Y, then the peers may exit
+        cluster_sync_all();
+        if (krank == 0 && warp >= 2 && warp < 6) {
+            const int jl = (warp & 3) * 32 + lane;
+            const int64_t col = (int64_t)tile0 * BM + jl;
+            const int rows = (int)(ep.M < NT ? ep.M : NT);
+            for (int t0 = 0; t0 < rows; t0 += 16) {
+                // 16 rows at a time: each rank's 16 loads are issued together
+                float y[16], v[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) y[t] = partial[(t0 + t) * BM + jl];
+                for (int r = 1; r < split; ++r) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) v[t] = ld_shared_cluster_f32(&partial[(t0 + t) * BM + jl], (uint32_t)r);
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) y[t] += v[t];
+                }
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    if (t0 + t < rows) {
+                        const int64_t idx = (int64_t)(t0 + t) * ep.N + col;
+                        if (ep.y_fp32) static_cast<float*>(ep.Y)[idx] = y[t];
+                        else           static_cast<__nv_bfloat16*>(ep.Y)[idx] = __float2bfloat16_rn(y[t]);
+                    }
+                }
+            }
+        }
+        cluster_sync_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -764,11 +810,28 @@ cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     }
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
     const int ntiles = p.N / BN;
-    const int grid = std::max(1, std::min(ntiles, std::max(1, sms)));
-    decode_kernel<FMT, ONE, NT><<<grid, kThreads, smem, s>>>(
-        tw, tb, tr, static_cast<const uint8_t*>(p.w_scales), static_cast<const uint8_t*>(p.bb_scales),
-        static_cast<const uint8_t*>(p.rs_scales), p.K, ep, ntiles);
-    return cudaGetLastError();
+    const int nk = p.K / BK;
+    // fewer tiles than SMs: clusters of `split` CTAs share a tile along K,
+    // each keeping at least 8 k-steps (shorter ranges do not pay for the
+    // cluster's setup and reduction)
+    int split = std::max(1, std::min(std::min(8, nk / 8), std::max(1, sms) / ntiles));
+    const int grid = split > 1 ? ntiles * split : std::max(1, std::min(ntiles, std::max(1, sms)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = split > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<FMT, ONE, NT>, tw, tb, tr,
+                              static_cast<const uint8_t*>(p.w_scales),
+                              static_cast<const uint8_t*>(p.bb_scales),
+                              static_cast<const uint8_t*>(p.rs_scales), p.K, ep, ntiles, split);
 }
 
 template <int FMT, int NT>

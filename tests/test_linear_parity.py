@@ -99,6 +99,9 @@ SHAPES = [
     (64, 256, 2048, "nvfp4"),
     (40, 128, 512, "mxfp4"),
     (1, 1024, 4096, "mxfp4"),
+    # K long enough that clusters of 4 and 8 CTAs split each tile along K
+    (5, 256, 8192, "nvfp4"),
+    (1, 128, 16384, "nvfp4"),
 ]
 
 
