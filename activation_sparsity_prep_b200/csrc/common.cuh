@@ -236,12 +236,6 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                  :: "r"(smem_u32(bar)) : "memory");
 }
 
-// Shared-memory -> tensor-memory copy of one 32-row x 16-byte scale atom,
-// replicated into all four 32-lane quarters.
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
-                 :: "r"(taddr), "l"(sdesc) : "memory");
-}
 
 // D(tmem) (+)= A(smem) x B(smem)^T, FP4 E2M1 operands, E4M3 scale per 16.
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -290,13 +284,9 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         : "r"(taddr));
 }
 
-// 32 lanes x 4 consecutive 32-bit columns from 4 registers per thread.
-__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
-                 :: "r"(taddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
 
-// 8 or 16 consecutive columns per lane in one store (two or four uint4).
+// 32 lanes x 8 or 16 consecutive 32-bit columns per lane in one store (two
+// or four uint4 per thread).
 __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint4 (&v)[2]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
                  :: "r"(taddr), "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w),
@@ -338,15 +328,5 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Descriptor of a 32-row x 16-byte scale atom (no swizzle, rows 16 B apart,
-// 8-row core matrices 128 B apart).
-__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
-    d |= (uint64_t)0 << 16;
-    d |= (uint64_t)(128u >> 4) << 32;
-    d |= (uint64_t)1 << 46;
-    return d;
-}
 
 }  // namespace sharq
