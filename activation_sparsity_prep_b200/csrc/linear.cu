@@ -119,11 +119,15 @@ struct SchedTables {
     int tpre[kMaxExperts + 1];   // tile prefix
 };
 
-// The grouped form uses the scheduler tables; the plain form uses the same
-// bytes as four 2 KiB epilogue staging buffers (one per epilogue warp).
+// Grouped form: the scheduler tables and one 1 KiB epilogue staging buffer
+// per epilogue warp.  Plain form (no tables): one 2 KiB staging buffer per
+// epilogue warp over the same bytes.
 union SchedSmem {
-    SchedTables t;
-    uint8_t stage[4][2048];
+    struct {
+        SchedTables t;
+        alignas(16) uint8_t stage[4][1024];
+    } g;
+    uint8_t stage2[4][2048];
 };
 
 __device__ __forceinline__ int ceil128(int x) { return (x + 127) >> 7; }
@@ -139,7 +143,7 @@ __device__ void sched_prepare(const Sched& sc, SchedSmem* sm) {
             int cnt = 0;
             if (e < sc.E) {
                 const int o0 = sc.offsets[e], o1 = sc.offsets[e + 1];
-                sm->t.off[e] = o0;
+                sm->g.t.off[e] = o0;
                 cnt = o1 - o0;
             }
             int pr = ceil128(cnt) * 128, tl = ceil128(cnt) * sc.nt_count;
@@ -149,20 +153,20 @@ __device__ void sched_prepare(const Sched& sc, SchedSmem* sm) {
                 int vp = __shfl_up_sync(0xffffffffu, ip, o), vt = __shfl_up_sync(0xffffffffu, it, o);
                 if (lane >= o) { ip += vp; it += vt; }
             }
-            if (e < sc.E) { sm->t.poff[e] = carry_p + ip - pr; sm->t.tpre[e] = carry_t + it - tl; }
+            if (e < sc.E) { sm->g.t.poff[e] = carry_p + ip - pr; sm->g.t.tpre[e] = carry_t + it - tl; }
             carry_p += __shfl_sync(0xffffffffu, ip, 31);
             carry_t += __shfl_sync(0xffffffffu, it, 31);
         }
         if (lane == 0) {
-            sm->t.off[sc.E] = sc.offsets[sc.E];
-            sm->t.poff[sc.E] = carry_p;
-            sm->t.tpre[sc.E] = carry_t;
+            sm->g.t.off[sc.E] = sc.offsets[sc.E];
+            sm->g.t.poff[sc.E] = carry_p;
+            sm->g.t.tpre[sc.E] = carry_t;
         }
     }
 }
 
 __device__ __forceinline__ int sched_count(const Sched& sc, const SchedSmem* sm) {
-    return sc.grouped ? sm->t.tpre[sc.E] : sc.mt_count * sc.nt_count;
+    return sc.grouped ? sm->g.t.tpre[sc.E] : sc.mt_count * sc.nt_count;
 }
 
 __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem* sm, int t) {
@@ -181,17 +185,17 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
     int lo = 0, hi = sc.E;                          // largest e with tpre[e] <= t
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (sm->t.tpre[mid] <= t) lo = mid; else hi = mid;
+        if (sm->g.t.tpre[mid] <= t) lo = mid; else hi = mid;
     }
     const int e = lo;
-    const int cnt = sm->t.off[e + 1] - sm->t.off[e];
+    const int cnt = sm->g.t.off[e + 1] - sm->g.t.off[e];
     const int mtn = ceil128(cnt);
-    const int local = t - sm->t.tpre[e];
+    const int local = t - sm->g.t.tpre[e];
     const int nt = local / mtn, mt = local - nt * mtn;
-    ti.a_row = sm->t.poff[e] + (int64_t)mt * 128;
+    ti.a_row = sm->g.t.poff[e] + (int64_t)mt * 128;
     ti.w_row = (int64_t)e * sc.N + (int64_t)nt * 128;
     ti.w_sf = (int64_t)e * sc.w_sf_stride + (int64_t)nt * (sc.nsf / 4) * 512;
-    ti.y_row = sm->t.off[e] + (int64_t)mt * 128;
+    ti.y_row = sm->g.t.off[e] + (int64_t)mt * 128;
     ti.rows = min(128, cnt - mt * 128);
     ti.col = nt * 128;
     ti.e = e;
@@ -410,21 +414,36 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+                // Stage the tile in shared memory so that every store
+                // instruction writes whole 32-byte sectors of several rows
+                // instead of 32 rows x 16 bytes.  Rows past ti.rows (the
+                // matrix end, or the next expert's rows in the grouped form)
+                // are not written.
+                const int64_t wrow0 = ti.y_row + q * 32;
+                __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(ep.Y);
                 if (sc.grouped) {
-                    // rows past the group belong to the next expert: masked row stores
-                    if (row_ok) {
-                        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(ep.Y) + row * ep.N + col0;
+                    // 32 rows x 16 columns at a time: 16 rows x 32 bytes per store
+                    uint8_t* stg = ssm->g.stage[q];
 #pragma unroll
-                        for (int i = 0; i < BN / 8; ++i)
-                            *reinterpret_cast<uint4*>(y + 8 * i) =
-                                make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+                    for (int hc = 0; hc < BN / 16; ++hc) {
+#pragma unroll
+                        for (int p = 0; p < 2; ++p)
+                            *reinterpret_cast<uint4*>(stg + lane * 32 + 16 * (p ^ ((lane >> 2) & 1))) =
+                                make_uint4(out[hc * 8 + 4 * p], out[hc * 8 + 4 * p + 1],
+                                           out[hc * 8 + 4 * p + 2], out[hc * 8 + 4 * p + 3]);
+                        __syncwarp();
+#pragma unroll
+                        for (int st = 0; st < 2; ++st) {
+                            const int r = 16 * st + (lane >> 1), p = lane & 1;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 32 + 16 * (p ^ ((r >> 2) & 1)));
+                            if (q * 32 + r < ti.rows)
+                                *reinterpret_cast<uint4*>(yb + (wrow0 + r) * ep.N + col0 + hc * 16 + p * 8) = v;
+                        }
+                        __syncwarp();
                     }
                 } else {
-                    // Stage each 32-row x 32-column chunk in shared memory so
-                    // that every store instruction writes 8 rows x 64
-                    // contiguous bytes instead of 32 rows x 16 bytes.
-                    uint8_t* stg = ssm->stage[q];
-                    const int64_t wrow0 = ti.y_row + q * 32;
+                    // 32 rows x 32 columns at a time: 8 rows x 64 bytes per store
+                    uint8_t* stg = ssm->stage2[q];
 #pragma unroll
                     for (int cc = 0; cc < BN / 32; ++cc) {
 #pragma unroll
@@ -438,8 +457,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                             const int r = 8 * st8 + (lane >> 2), p = lane & 3;
                             const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (p ^ (r & 3)));
                             if (q * 32 + r < ti.rows)
-                                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(ep.Y) +
-                                                          (wrow0 + r) * ep.N + col0 + cc * 32 + p * 8) = v;
+                                *reinterpret_cast<uint4*>(yb + (wrow0 + r) * ep.N + col0 + cc * 32 + p * 8) = v;
                         }
                         __syncwarp();
                     }
@@ -879,10 +897,10 @@ moe_gather_kernel(const uint8_t* __restrict__ bb_codes, const uint8_t* __restric
         int lo = 0, hi = sc.E;                      // expert of row t
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (ssm.t.off[mid] <= t) lo = mid; else hi = mid;
+            if (ssm.g.t.off[mid] <= t) lo = mid; else hi = mid;
         }
         const int64_t src = row_index ? (int64_t)row_index[t] : t;
-        const int64_t dst = ssm.t.poff[lo] + (t - ssm.t.off[lo]);
+        const int64_t dst = ssm.g.t.poff[lo] + (t - ssm.g.t.off[lo]);
         const uint4* sb = reinterpret_cast<const uint4*>(bb_codes + src * row_bytes);
         const uint4* sr = reinterpret_cast<const uint4*>(rs_codes + src * row_bytes);
         uint4* db = reinterpret_cast<uint4*>(gb_codes + dst * row_bytes);
