@@ -28,6 +28,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 namespace sharq {
 namespace {
 
@@ -732,16 +734,29 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once (thread-safe static initialisation).
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static const EncodeTiledFn fn = [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
+}
+
+// Per-device "attribute already set" flags; setting an attribute twice is
+// harmless, so concurrent first calls only need the flag itself to be atomic.
+template <class Fn>
+cudaError_t set_smem_once(std::atomic<bool> (&done)[64], Fn kernel, size_t bytes) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev < 64) done[dev].store(true, std::memory_order_release);
+    return e;
 }
 
 // 2-D uint8 map over a [rows, row_bytes] code matrix, box 128 bytes x box_rows,
@@ -765,16 +780,8 @@ size_t linear_smem_bytes() {
 
 template <int FMT, bool ONE>
 cudaError_t ensure_smem_attr() {
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(linear_kernel<FMT, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)linear_smem_bytes<FMT>());
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[dev] = true;
-    }
-    return cudaSuccess;
+    static std::atomic<bool> done[64];
+    return set_smem_once(done, linear_kernel<FMT, ONE>, linear_smem_bytes<FMT>());
 }
 
 // A_rows: rows of the activation operands (gathered and padded for the
@@ -817,15 +824,8 @@ cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
         !make_code_map(&tr, p.rs_codes, p.M, p.K / 2, NT))
         return cudaErrorInvalidValue;
     const size_t smem = D::S * D::kStageStride + sizeof(DecBarriers<D::S>) + 1024;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<FMT, ONE, NT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[dev] = true;
-    }
+    static std::atomic<bool> done[64];
+    if (cudaError_t e = set_smem_once(done, decode_kernel<FMT, ONE, NT>, smem); e != cudaSuccess) return e;
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
     const int ntiles = p.N / BN;
     const int nk = p.K / BK;

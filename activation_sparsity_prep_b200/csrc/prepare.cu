@@ -24,6 +24,8 @@
 
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 namespace sharq {
 
 unsigned take_status_prepare() { return take_tu_status(); }
@@ -640,12 +642,13 @@ prepare_kernel(PrepArgs a) {
 template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false, bool LN = false>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN>;
-    static int blocks_per_sm = 0;          // same for every device of one architecture
+    // same for every device of one architecture; a repeated query is harmless
+    static std::atomic<int> cached{0};
+    int blocks_per_sm = cached.load(std::memory_order_relaxed);
     if (blocks_per_sm == 0) {
-        int b = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kfn, kThreads, 0);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kfn, kThreads, 0);
         if (e != cudaSuccess) return e;
-        blocks_per_sm = b;
+        cached.store(blocks_per_sm, std::memory_order_relaxed);
     }
     // Enough warps for one row each in phase 1 and about four 32-block
     // groups each in phases 2 and 3, capped at what is resident.
