@@ -21,16 +21,17 @@ def _outputs(P):
     return [P.bb_codes, P.bb_scales, P.bb_tscale, P.rs_codes, P.rs_scales, P.rs_tscale, P.mask]
 
 
-@pytest.mark.parametrize("M,K,gamma,fmt", [(300, 4096, True, "nvfp4"), (17, 768, False, "nvfp4"),
-                                           (129, 1024, True, "mxfp4")])
-def test_noalloc_matches_workspace_entry_point_on_two_calls(M, K, gamma, fmt):
+@pytest.mark.parametrize("M,K,gamma,fmt,rs", [(300, 4096, True, "nvfp4", "own"), (17, 768, False, "nvfp4", "own"),
+                                              (129, 1024, True, "mxfp4", "own"),
+                                              (200, 2048, True, "nvfp4", "shared")])
+def test_noalloc_matches_workspace_entry_point_on_two_calls(M, K, gamma, fmt, rs):
     L = sq.load_sharq_ops()
     X = torch.from_numpy(wl.activation("laplace_outlier", 41, M, M, K)).view(torch.bfloat16).cuda()
     g = torch.from_numpy(wl.gamma_ones(K)).view(torch.bfloat16).cuda() if gamma else None
-    ref = sq.prepare(X, g, wl.EPS, 2, 4, fmt, want_mask=True)
+    ref = sq.prepare(X, g, wl.EPS, 2, 4, fmt, want_mask=True, residual_scale=rs)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
-        out = sq.Prepared.empty(M, K, 2, 4, fmt, want_mask=True)
+        out = sq.Prepared.empty(M, K, 2, 4, fmt, want_mask=True, residual_scale=rs)
         for t in _outputs(out):
             t.fill_(0xA5 if t.dtype == torch.uint8 else 7.0)      # poison
         c = out._c()
