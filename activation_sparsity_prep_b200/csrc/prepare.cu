@@ -11,10 +11,11 @@
 //   phase 3  residual codes/scales with G_r
 // One persistent cooperative launch runs the three phases.  In phase 1 each
 // warp owns whole rows, lane l reading the 16-byte chunks l, l+32, ... of a
-// row, which is also the fixed fp32 reduction order of the RMS sum; phases 2
-// and 3 spread (row, 256-element segment) items over every warp.  MXFP4 has
-// no tensor scale, so its backbone and residual are produced in one pass
-// (after the RMS barrier when there is a norm).
+// row, which is also the fixed fp32 reduction order of the RMS sum; without
+// a norm, phase 1 is a plain maximum over the whole tensor, spread over every
+// lane.  Phases 2 and 3 spread (row, 256-element segment) items over every
+// warp.  MXFP4 has no tensor scale, so its backbone and residual are produced
+// in one pass (after the RMS barrier when there is a norm).
 //
 // Every floating-point step is one correctly rounded fp32 operation
 // (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn, no contraction), so the
@@ -339,106 +340,108 @@ prepare_kernel(PrepArgs a) {
     float* rinv_ws = ws_rinv(a.ws);
 
     // ---------------- phase 1: rinv per row, A_b = max |y| ----------------
-    // One warp per row: lane l adds the squares of chunks l, l+32, ... in k
-    // order (the fixed reduction order), eight chunk loads in flight per lane.
     float amax = 0.0f;
-    if (HAS_GAMMA || FMT == 0) {
-        for (int64_t row = gwarp; row < M; row += nwarps) {
-            const uint16_t* xr = a.X + row * K;
-            float rinv = 1.0f, mu = 0.0f;
-            if (HAS_GAMMA) {
-                // One pass in the fixed order: lane l adds f(x) over chunks
-                // l, l+32, ... element by element, then the xor butterfly.
-                auto row_sum = [&](auto f) {
-                    float acc = 0.0f;
-                    for (int c0 = lane; c0 < nchunk; c0 += 256) {
-                        uint4 v[8];
+    if (FMT == 0 && !HAS_GAMMA) {
+        // y = x, and A_b = max |x| needs no row structure: lane i of the
+        // grid reads chunks i, i + L, ..., i + 15L (L = lanes in the grid),
+        // sixteen loads in flight, then the next 16L chunks.  The magnitude
+        // order of bf16 values is the integer order of their bits with the
+        // sign cleared.
+        const int64_t nch = M * (int64_t)nchunk;
+        const int64_t L = nwarps * 32;
+        uint32_t m2 = 0;
+        for (int64_t c0 = gwarp * 32 + lane; c0 < nch; c0 += 16 * L) {
+            uint4 v[16];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+            for (int u = 0; u < 16; ++u)
+                if (c0 + u * L < nch) v[u] = ld_nc_v4(a.X + (c0 + u * L) * 8);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            if (c0 + 32 * u < nchunk) {
-                                float x[8];
-                                unpack_bf16x8(v[u], x);
-#pragma unroll
-                                for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, f(x[t]));
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1)
-                        acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
-                    return acc;
-                };
-                if (LN) {
-                    // LayerNorm: mean, then the centred squares (two passes)
-                    mu = __fdiv_rn(row_sum([](float x) { return x; }), (float)K);
-                    const float var = __fdiv_rn(row_sum([mu](float x) {
-                        const float d = __fsub_rn(x, mu);
-                        return __fmul_rn(d, d);
-                    }), (float)K);
-                    rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
-                    if (lane == 0) { rinv_ws[row] = rinv; rinv_ws[M + row] = mu; }
-                } else {
-                    const float ms = __fdiv_rn(row_sum([](float x) { return __fmul_rn(x, x); }), (float)K);
-                    rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
-                    if (lane == 0) rinv_ws[row] = rinv;
+            for (int u = 0; u < 16; ++u) {
+                if (c0 + u * L < nch) {
+                    m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
+                    m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
+                    m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
+                    m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
                 }
             }
+        }
+        amax = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    } else if (HAS_GAMMA) {
+        // One warp per row.  rinv: lane l adds f(x) over chunks l, l+32, ...
+        // element by element in k order, then the xor butterfly -- the fixed
+        // reduction order.  Then (NVFP4) the row's max |y|.  Eight chunk
+        // loads in flight per lane (four per operand for LayerNorm's max).
+        for (int64_t row = gwarp; row < M; row += nwarps) {
+            const uint16_t* xr = a.X + row * K;
+            auto row_sum = [&](auto f) {
+                float acc = 0.0f;
+                for (int c0 = lane; c0 < nchunk; c0 += 256) {
+                    uint4 v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (c0 + 32 * u < nchunk) {
+                            float x[8];
+                            unpack_bf16x8(v[u], x);
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, f(x[t]));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1)
+                    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+                return acc;
+            };
+            float rinv, mu = 0.0f;
+            if (LN) {
+                // LayerNorm: mean, then the centred squares (two passes)
+                mu = __fdiv_rn(row_sum([](float x) { return x; }), (float)K);
+                const float var = __fdiv_rn(row_sum([mu](float x) {
+                    const float d = __fsub_rn(x, mu);
+                    return __fmul_rn(d, d);
+                }), (float)K);
+                rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+                if (lane == 0) { rinv_ws[row] = rinv; rinv_ws[M + row] = mu; }
+            } else {
+                const float ms = __fdiv_rn(row_sum([](float x) { return __fmul_rn(x, x); }), (float)K);
+                rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+                if (lane == 0) rinv_ws[row] = rinv;
+            }
             if (FMT == 0) {
-                if (HAS_GAMMA) {
-                    for (int c0 = lane; c0 < nchunk; c0 += 128) {
-                        uint4 v[4], g[4], bt[LN ? 4 : 1];
+                constexpr int D = LN ? 4 : 8;   // LayerNorm also streams beta
+                for (int c0 = lane; c0 < nchunk; c0 += 32 * D) {
+                    uint4 v[D], g[D], bt[LN ? D : 1];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            if (c0 + 32 * u < nchunk) {
-                                v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
-                                g[u] = ld_nc_v4(a.gamma + (int64_t)(c0 + 32 * u) * 8);
-                                if (LN && has_beta) bt[u] = ld_nc_v4(a.beta + (int64_t)(c0 + 32 * u) * 8);
-                            }
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            if (c0 + 32 * u < nchunk) {
-                                float y[8], gg[8];
-                                unpack_bf16x8(v[u], y);
-                                unpack_bf16x8(g[u], gg);
-#pragma unroll
-                                for (int t = 0; t < 8; ++t) {
-                                    const float xv = LN ? __fsub_rn(y[t], mu) : y[t];
-                                    y[t] = __fmul_rn(__fmul_rn(xv, rinv), gg[t]);
-                                }
-                                if (LN && has_beta) {
-                                    float bb[8];
-                                    unpack_bf16x8(bt[u], bb);
-#pragma unroll
-                                    for (int t = 0; t < 8; ++t) y[t] = __fadd_rn(y[t], bb[t]);
-                                }
-                                amax = fmaxf(amax, amax8(y));
-                            }
+                    for (int u = 0; u < D; ++u) {
+                        if (c0 + 32 * u < nchunk) {
+                            v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+                            g[u] = ld_nc_v4(a.gamma + (int64_t)(c0 + 32 * u) * 8);
+                            if (LN && has_beta) bt[u] = ld_nc_v4(a.beta + (int64_t)(c0 + 32 * u) * 8);
                         }
                     }
-                } else {
-                    // y = x: the magnitude order of bf16 values is the integer
-                    // order of their bits with the sign cleared.
-                    uint32_t m2 = 0;
-                    for (int c0 = lane; c0 < nchunk; c0 += 256) {
-                        uint4 v[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
+                    for (int u = 0; u < D; ++u) {
+                        if (c0 + 32 * u < nchunk) {
+                            float y[8], gg[8];
+                            unpack_bf16x8(v[u], y);
+                            unpack_bf16x8(g[u], gg);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            if (c0 + 32 * u < nchunk) {
-                                m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
-                                m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
-                                m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
-                                m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+                            for (int t = 0; t < 8; ++t) {
+                                const float xv = LN ? __fsub_rn(y[t], mu) : y[t];
+                                y[t] = __fmul_rn(__fmul_rn(xv, rinv), gg[t]);
                             }
+                            if (LN && has_beta) {
+                                float bb[8];
+                                unpack_bf16x8(bt[u], bb);
+#pragma unroll
+                                for (int t = 0; t < 8; ++t) y[t] = __fadd_rn(y[t], bb[t]);
+                            }
+                            amax = fmaxf(amax, amax8(y));
                         }
                     }
-                    amax = fmaxf(amax, fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u)));
                 }
             }
         }
