@@ -333,6 +333,64 @@ def moe_linear(prep: Prepared, row_index: np.ndarray, offsets: np.ndarray,
     return Y
 
 
+# ------------------------------------------------ producer-fused MLP ----
+# SharQ paper, Abstract: the preparation is one operator in front of each
+# FP4 linear.  For a SwiGLU MLP the down projection's input is
+# silu(gate) * up, both halves of the gate+up linear; the fused form computes
+# it in that linear's epilogue.  SwiGLU itself is the standard gated unit
+# (Shazeer, "GLU Variants Improve Transformer", 2020): silu(x W_g) * (x W_u).
+
+GATE_UP_BLOCK = 64
+
+
+def interleave_gate_up(W_gate: np.ndarray, W_up: np.ndarray) -> np.ndarray:
+    """[I, K] gate and up weights -> the [2I, K] layout of the fused linear:
+    rows 128t .. 128t+63 are gate rows 64t .. 64t+63 and rows
+    128t+64 .. 128t+127 the up rows with the same indices, so that every
+    128-row output tile holds 64 gate columns and their 64 up columns."""
+    I, K = W_gate.shape
+    if W_up.shape != (I, K) or I % GATE_UP_BLOCK:
+        raise ValueError("gate and up must both be [I, K] with I a multiple of 64")
+    out = np.empty((2 * I, K), dtype=W_gate.dtype)
+    for t in range(I // GATE_UP_BLOCK):
+        out[128 * t:128 * t + 64] = W_gate[64 * t:64 * t + 64]
+        out[128 * t + 64:128 * t + 128] = W_up[64 * t:64 * t + 64]
+    return out
+
+
+def silu(x) -> np.ndarray:
+    """x * sigmoid(x) = x / (1 + e^-x) in fp64 (e^-x overflows to inf for
+    x < -709, giving -0)."""
+    x = np.asarray(x, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-x))
+
+
+def _deinterleave(Y: np.ndarray):
+    """Columns of a [R, 2I] gate+up output -> (gate [R, I], up [R, I])."""
+    R, N = Y.shape
+    t = np.arange(N // 2) // GATE_UP_BLOCK
+    j = np.arange(N // 2) % GATE_UP_BLOCK
+    return Y[:, 128 * t + j], Y[:, 128 * t + 64 + j]
+
+
+def swiglu_linear(prep: Prepared, w: Quantized, rows: Optional[np.ndarray] = None) -> np.ndarray:
+    """The two-path linear over the interleaved gate+up weight followed by
+    the SwiGLU gate, in fp64: H[:, 64t + j] = silu(Y[:, 128t + j]) *
+    Y[:, 128t + 64 + j].  Returns [R, I]."""
+    g, u = _deinterleave(linear(prep, w, rows))
+    return silu(g) * u
+
+
+def swiglu_parts(prep: Prepared, w: Quantized, rows: Optional[np.ndarray] = None):
+    """(gate, up, |gate| bound, |up| bound) of the fused linear in fp64: the
+    two halves of the linear and their magnitude sums (linear_abs), from
+    which a test derives the rounding bound of an fp32 evaluation."""
+    g, u = _deinterleave(linear(prep, w, rows))
+    ga, ua = _deinterleave(linear_abs(prep, w, rows))
+    return g, u, ga, ua
+
+
 def bf16_rne_from_f64(Y: np.ndarray) -> np.ndarray:
     """RNE(Y64) to bf16 bits, the reference for the bf16 output (fp64 -> bf16
     in one rounding, done exactly through the neighbouring bf16 values)."""
