@@ -89,6 +89,10 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_prepare_layernorm.restype = I
         L.sharq_linear.argtypes = [ctypes.POINTER(_Prepared), ctypes.POINTER(_Weight), P, I, P]
         L.sharq_linear.restype = I
+        L.sharq_linear_swiglu.argtypes = [ctypes.POINTER(_Prepared), ctypes.POINTER(_Weight), P, P, P]
+        L.sharq_linear_swiglu.restype = I
+        L.sharq_prepare_amax.argtypes = [P, P, ctypes.POINTER(_Prepared), P, SZ, P]
+        L.sharq_prepare_amax.restype = I
         L.sharq_moe_workspace_bytes.argtypes = [I64, I, I, I]
         L.sharq_moe_workspace_bytes.restype = SZ
         L.sharq_moe_linear.argtypes = [ctypes.POINTER(_Prepared), P, P, I, I64,
@@ -288,6 +292,48 @@ def linear(x: Prepared, w: Weight, out_fp32: bool = False, out=None, stream=None
     _check("sharq_linear", L.sharq_linear(ctypes.byref(cx), ctypes.byref(cw), Y.data_ptr(),
                                           1 if out_fp32 else 0, _stream(stream)))
     return Y
+
+
+def interleave_gate_up(W_gate, W_up):
+    """[I, K] gate and up weights (bf16 tensors) -> the [2I, K] layout that
+    linear_swiglu expects: per 128 rows, 64 gate rows then the 64 up rows with
+    the same indices.  An offline layout step of the weight, done once."""
+    import torch
+    I, K = W_gate.shape
+    if tuple(W_up.shape) != (I, K) or I % 64:
+        raise ValueError("gate and up must both be [I, K] with I a multiple of 64")
+    return torch.stack((W_gate.reshape(I // 64, 64, K), W_up.reshape(I // 64, 64, K)), 1).reshape(2 * I, K)
+
+
+def linear_swiglu(x: Prepared, w: Weight, out=None, amax=None, stream=None):
+    """Gate+up linear with the SwiGLU epilogue: returns (H bf16 [M, w.N/2],
+    amax fp32 [1] = max |H|), for w quantised from interleave_gate_up(...)."""
+    import torch
+    L = load_sharq_ops()
+    dev = x.bb_codes.device
+    H = out if out is not None else torch.empty((x.M, w.N // 2), dtype=torch.bfloat16, device=dev)
+    a = amax if amax is not None else torch.empty((1,), dtype=torch.float32, device=dev)
+    cx, cw = x._c(), w._c()
+    _check("sharq_linear_swiglu", L.sharq_linear_swiglu(ctypes.byref(cx), ctypes.byref(cw), H.data_ptr(),
+                                                        a.data_ptr(), _stream(stream)))
+    return H, a
+
+
+def prepare_amax(X, amax, n: int = 2, m: int = 4, fmt="nvfp4", want_mask: bool = False,
+                 out: Optional[Prepared] = None, ws=None, stream=None, residual_scale="own") -> Prepared:
+    """prepare() of a no-norm input whose max |X| the producer has already
+    taken (amax: fp32 [1] device tensor, e.g. from linear_swiglu)."""
+    L = load_sharq_ops()
+    M, K = X.shape
+    f = _fmt(fmt)
+    p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
+                                                   residual_scale=residual_scale)
+    ws = _workspace(M, K, f, ws, X.device)
+    cp = p._c()
+    _check("sharq_prepare_amax",
+           L.sharq_prepare_amax(X.data_ptr(), amax.data_ptr(), ctypes.byref(cp), ws.data_ptr(),
+                                ws.numel(), _stream(stream)))
+    return p
 
 
 def moe_workspace_bytes(T: int, E: int, K: int, fmt="nvfp4") -> int:

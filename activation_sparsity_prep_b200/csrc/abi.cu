@@ -88,7 +88,7 @@ sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_weight* out, 
 
 static sharq_status prepare_common(const void* X_bf16, const void* gamma_bf16, const void* beta_bf16,
                                    bool layernorm, float eps, const sharq_prepared* out, void* ws,
-                                   size_t ws_bytes, void* stream) {
+                                   size_t ws_bytes, void* stream, const float* amax = nullptr) {
     if (!out || !ws) return SHARQ_ERR_INVALID_ARG;
     if (layernorm && out->M > 0 && !gamma_bf16) return SHARQ_ERR_INVALID_ARG;
     if (!aligned16(beta_bf16)) return SHARQ_ERR_INVALID_ARG;
@@ -113,7 +113,7 @@ static sharq_status prepare_common(const void* X_bf16, const void* gamma_bf16, c
     p.fmt = o.fmt; p.weight = false; p.residual_shared = o.residual_scale == SHARQ_RESIDUAL_SHARED;
     p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
     p.rs_codes = o.rs_codes; p.rs_scales = o.rs_scales; p.rs_tscale = o.rs_tscale;
-    p.mask = o.mask; p.ws = ws;
+    p.mask = o.mask; p.ws = ws; p.amax = amax;
     return cuda_status(sharq::launch_prepare(p, static_cast<cudaStream_t>(stream),
                                              sharq::device_sm_count()));
 }
@@ -127,6 +127,12 @@ sharq_status sharq_prepare_layernorm(const void* X_bf16, const void* gamma_bf16,
                                      float eps, const sharq_prepared* out, void* ws, size_t ws_bytes,
                                      void* stream) {
     return prepare_common(X_bf16, gamma_bf16, beta_bf16, true, eps, out, ws, ws_bytes, stream);
+}
+
+sharq_status sharq_prepare_amax(const void* X_bf16, const float* amax, const sharq_prepared* out,
+                                void* ws, size_t ws_bytes, void* stream) {
+    if (!amax || ((uintptr_t)amax & 3u)) return SHARQ_ERR_INVALID_ARG;
+    return prepare_common(X_bf16, nullptr, nullptr, false, 0.0f, out, ws, ws_bytes, stream, amax);
 }
 
 static sharq_status check_linear_args(const sharq_prepared* x, const sharq_weight* w, void* Y) {
@@ -157,6 +163,24 @@ sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w, void* 
     p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
     p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
     p.one_acc = x->fmt == SHARQ_MXFP4 || x->residual_scale == SHARQ_RESIDUAL_SHARED;
+    return cuda_status(sharq::launch_linear(p, static_cast<cudaStream_t>(stream),
+                                            sharq::device_sm_count()));
+}
+
+sharq_status sharq_linear_swiglu(const sharq_prepared* x, const sharq_weight* w, void* H,
+                                 float* h_amax, void* stream) {
+    sharq_status st = check_linear_args(x, w, H);
+    if (st != SHARQ_OK) return st;
+    if (!h_amax || ((uintptr_t)h_amax & 3u)) return SHARQ_ERR_INVALID_ARG;
+    if (x->M == 0)
+        return cuda_status(cudaMemsetAsync(h_amax, 0, sizeof(float), static_cast<cudaStream_t>(stream)));
+    sharq::LinearLaunch p{};
+    p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
+    p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
+    p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
+    p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = H; p.y_fp32 = 0;
+    p.one_acc = x->fmt == SHARQ_MXFP4 || x->residual_scale == SHARQ_RESIDUAL_SHARED;
+    p.swiglu = true; p.amax = h_amax;
     return cuda_status(sharq::launch_linear(p, static_cast<cudaStream_t>(stream),
                                             sharq::device_sm_count()));
 }

@@ -9,7 +9,11 @@
 //   acc_b += A_b x W^T,   acc_r += A_r x W^T.
 // The epilogue reads both accumulators back and writes
 //   Y = G_w * (G_b * acc_b + G_r * acc_r)
-// as bf16 (or fp32).  When the two tensor scales are equal by construction
+// as bf16 (or fp32).  The SwiGLU form (the gate+up projection of an MLP,
+// its weight rows interleaved 64 gate / 64 up per 128-row tile) writes
+// H = silu(gate) * up instead, half as many bf16 columns, and the maximum of
+// |H|: the next prepare's backbone amax, so that prepare skips its own
+// pass over H.  When the two tensor scales are equal by construction
 // (MXFP4, or a residual quantised against the backbone's tensor scale) both
 // MMAs accumulate into one accumulator, Y = G_w * G_b * acc, and the two
 // tensor-memory accumulators serve as a double buffer instead: the next
@@ -83,7 +87,16 @@ struct EpiArgs {
     int64_t M;
     int N;
     int y_fp32;
+    uint32_t* amax;    // SwiGLU form: max |H| as fp32 bits (zeroed before the launch)
 };
+
+// silu(g) = g / (1 + e^-g) in fp32 with the fast exponential and divide
+// (relative error within (5 + 1.2 |g|) 2^-23 while 1 + e^-g < 2^126, i.e.
+// g > -87; below that the quotient is 0, against a true |silu| < 1e-36).
+// The correctly rounded forms cost about 6 % of the gate+up linear's time.
+__device__ __forceinline__ float silu_f32(float g) {
+    return __fdividef(g, 1.0f + __expf(-g));
+}
 
 // One output tile of the (plain or grouped) problem.
 struct TileInfo {
@@ -209,7 +222,7 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
 // thread waits only until the epilogue has copied the previous tile's two
 // accumulators out of tensor memory, so the epilogue's global stores overlap
 // the next tile's MMAs.
-template <int FMT, bool ONE>
+template <int FMT, bool ONE, bool SW>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_r,
               const __grid_constant__ CUtensorMap tm_w, const uint8_t* __restrict__ sf_b,
@@ -355,6 +368,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
         const int q = warp & 3;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const float gbb = *ep.bb_tscale, grr = *ep.rs_tscale;
+        uint32_t hmax = 0;      // SwiGLU: running max of |H| as two bf16 magnitudes
         uint32_t tc = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
             const TileInfo ti = sched_tile(sc, ssm, tile);
@@ -370,7 +384,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             if (!ok) break;
             const uint32_t src_b = ONE ? tmem + buf * BN : t_acc_b;
             const int64_t col0 = ti.col;
-            if (ep.y_fp32) {
+            if (!SW && ep.y_fp32) {
 #pragma unroll 1
                 for (int cc = 0; cc < BN / 32; ++cc) {
                     uint32_t vb[32], vr[32];
@@ -394,28 +408,64 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
             } else {
-                // drain both accumulators into 64 packed bf16x2 registers, hand
-                // the tensor memory back, then store
-                uint32_t out[BN / 2];
+                // drain the accumulators into packed bf16x2 registers (64 for
+                // Y, 32 for H), hand the tensor memory back, then store
+                constexpr int kOutCols = SW ? BN / 2 : BN;
+                uint32_t out[kOutCols / 2];
+                if constexpr (SW) {
+                    // columns j and 64 + j of the tile: gate and up of feature j.
+                    // Drain all 128 values first and hand the tensor memory back,
+                    // so the next tile's MMAs run under the SwiGLU arithmetic.
+                    float gv[BN / 2], uv[BN / 2];
 #pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) {
-                    uint32_t vb[32], vr[32];
-                    tmem_ld_32x32b_x32(src_b + lane_off + cc * 32, vb);
-                    if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
-                    tmem_ld_wait();
+                    for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) {
-                        float lo = ONE ? gb * __uint_as_float(vb[2 * h])
-                                       : gb * __uint_as_float(vb[2 * h]) + gr * __uint_as_float(vr[2 * h]);
-                        float hi = ONE ? gb * __uint_as_float(vb[2 * h + 1])
-                                       : gb * __uint_as_float(vb[2 * h + 1]) + gr * __uint_as_float(vr[2 * h + 1]);
-                        __nv_bfloat162 p2 = __floats2bfloat162_rn(lo, hi);
-                        out[cc * 16 + h] = *reinterpret_cast<uint32_t*>(&p2);
+                        for (int cc = 0; cc < 2; ++cc) {
+                            uint32_t vb[32], vr[32];
+                            const uint32_t c = half * (BN / 2) + cc * 32;
+                            tmem_ld_32x32b_x32(src_b + lane_off + c, vb);
+                            if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + c, vr);
+                            tmem_ld_wait();
+                            float* dst = half ? uv : gv;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                dst[cc * 32 + i] = ONE ? gb * __uint_as_float(vb[i])
+                                                       : gb * __uint_as_float(vb[i]) + gr * __uint_as_float(vr[i]);
+                        }
                     }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+#pragma unroll
+                    for (int h = 0; h < BN / 4; ++h) {
+                        const float h0 = __fmul_rn(silu_f32(gv[2 * h]), uv[2 * h]);
+                        const float h1 = __fmul_rn(silu_f32(gv[2 * h + 1]), uv[2 * h + 1]);
+                        __nv_bfloat162 p2 = __floats2bfloat162_rn(h0, h1);
+                        const uint32_t bits = *reinterpret_cast<uint32_t*>(&p2);
+                        out[h] = bits;
+                        if (row_ok) hmax = __vmaxu2(hmax, bits & 0x7FFF7FFFu);
+                    }
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < BN / 32; ++cc) {
+                        uint32_t vb[32], vr[32];
+                        tmem_ld_32x32b_x32(src_b + lane_off + cc * 32, vb);
+                        if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) {
+                            float lo = ONE ? gb * __uint_as_float(vb[2 * h])
+                                           : gb * __uint_as_float(vb[2 * h]) + gr * __uint_as_float(vr[2 * h]);
+                            float hi = ONE ? gb * __uint_as_float(vb[2 * h + 1])
+                                           : gb * __uint_as_float(vb[2 * h + 1]) + gr * __uint_as_float(vr[2 * h + 1]);
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(lo, hi);
+                            out[cc * 16 + h] = *reinterpret_cast<uint32_t*>(&p2);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
                 // Stage the tile in shared memory so that every store
                 // instruction writes whole 32-byte sectors of several rows
                 // instead of 32 rows x 16 bytes.  Rows past ti.rows (the
@@ -423,7 +473,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 // are not written.
                 const int64_t wrow0 = ti.y_row + q * 32;
                 __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(ep.Y);
-                if (sc.grouped) {
+                if (!SW && sc.grouped) {
                     // 32 rows x 16 columns at a time: 16 rows x 32 bytes per store
                     uint8_t* stg = ssm->g.stage[q];
 #pragma unroll
@@ -446,8 +496,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 } else {
                     // 32 rows x 32 columns at a time: 8 rows x 64 bytes per store
                     uint8_t* stg = ssm->stage2[q];
+                    const int64_t ldy = SW ? ep.N / 2 : ep.N;     // H has N/2 columns
+                    const int64_t ycol = SW ? col0 / 2 : col0;
 #pragma unroll
-                    for (int cc = 0; cc < BN / 32; ++cc) {
+                    for (int cc = 0; cc < kOutCols / 32; ++cc) {
 #pragma unroll
                         for (int p = 0; p < 4; ++p)
                             *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (p ^ (lane & 3))) =
@@ -459,12 +511,20 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                             const int r = 8 * st8 + (lane >> 2), p = lane & 3;
                             const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (p ^ (r & 3)));
                             if (q * 32 + r < ti.rows)
-                                *reinterpret_cast<uint4*>(yb + (wrow0 + r) * ep.N + col0 + cc * 32 + p * 8) = v;
+                                *reinterpret_cast<uint4*>(yb + (wrow0 + r) * ldy + ycol + cc * 32 + p * 8) = v;
                         }
                         __syncwarp();
                     }
                 }
             }
+        }
+        if (SW) {
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) hmax = __vmaxu2(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+            // the larger of the two bf16 magnitudes, as fp32 bits (non-negative
+            // floats order as unsigned integers)
+            const uint32_t m = max(hmax << 16, hmax & 0xFFFF0000u);
+            if (lane == 0 && m) atomicMax(ep.amax, m);
         }
     }
     tc_fence_before();
@@ -778,15 +838,15 @@ size_t linear_smem_bytes() {
     return kStages * Cfg<FMT>::kStageStride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
 }
 
-template <int FMT, bool ONE>
+template <int FMT, bool ONE, bool SW>
 cudaError_t ensure_smem_attr() {
     static std::atomic<bool> done[64];
-    return set_smem_once(done, linear_kernel<FMT, ONE>, linear_smem_bytes<FMT>());
+    return set_smem_once(done, linear_kernel<FMT, ONE, SW>, linear_smem_bytes<FMT>());
 }
 
 // A_rows: rows of the activation operands (gathered and padded for the
 // grouped form); W_rows: rows of the (stacked) weight.
-template <int FMT, bool ONE>
+template <int FMT, bool ONE, bool SW>
 cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const void* rs_codes,
                         const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
                         const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
@@ -795,11 +855,16 @@ cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const voi
         !make_code_map(&tr, rs_codes, A_rows, p.K / 2, BM) ||
         !make_code_map(&tw, p.w_codes, W_rows, p.K / 2, BN))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr<FMT, ONE>();
+    cudaError_t e = ensure_smem_attr<FMT, ONE, SW>();
     if (e != cudaSuccess) return e;
-    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
+    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32,
+               reinterpret_cast<uint32_t*>(p.amax)};
+    if (SW) {
+        e = cudaMemsetAsync(p.amax, 0, sizeof(float), s);
+        if (e != cudaSuccess) return e;
+    }
     const int grid = std::max(1, std::min(max_tiles, std::max(1, sms)));
-    linear_kernel<FMT, ONE><<<grid, kThreads, linear_smem_bytes<FMT>(), s>>>(
+    linear_kernel<FMT, ONE, SW><<<grid, kThreads, linear_smem_bytes<FMT>(), s>>>(
         tb, tr, tw, static_cast<const uint8_t*>(bb_scales), static_cast<const uint8_t*>(rs_scales),
         static_cast<const uint8_t*>(p.w_scales), p.K, ep, sc);
     return cudaGetLastError();
@@ -809,10 +874,15 @@ template <int FMT>
 cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void* rs_codes,
                         const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
                         const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
-    return p.one_acc ? launch_gemm_t<FMT, true>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows, p,
-                                               W_rows, sc, max_tiles, s, sms)
-                     : launch_gemm_t<FMT, false>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows, p,
-                                                W_rows, sc, max_tiles, s, sms);
+    if (p.swiglu)
+        return p.one_acc ? launch_gemm_t<FMT, true, true>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows,
+                                                          p, W_rows, sc, max_tiles, s, sms)
+                         : launch_gemm_t<FMT, false, true>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows,
+                                                           p, W_rows, sc, max_tiles, s, sms);
+    return p.one_acc ? launch_gemm_t<FMT, true, false>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows, p,
+                                                      W_rows, sc, max_tiles, s, sms)
+                     : launch_gemm_t<FMT, false, false>(bb_codes, bb_scales, rs_codes, rs_scales, A_rows, p,
+                                                       W_rows, sc, max_tiles, s, sms);
 }
 
 template <int FMT, bool ONE, int NT>
@@ -826,7 +896,7 @@ cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     const size_t smem = D::S * D::kStageStride + sizeof(DecBarriers<D::S>) + 1024;
     static std::atomic<bool> done[64];
     if (cudaError_t e = set_smem_once(done, decode_kernel<FMT, ONE, NT>, smem); e != cudaSuccess) return e;
-    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32};
+    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32, nullptr};
     const int ntiles = p.N / BN;
     const int nk = p.K / BK;
     // fewer tiles than SMs: clusters of `split` CTAs share a tile along K,
@@ -859,10 +929,13 @@ cudaError_t launch_decode_nt(const LinearLaunch& p, cudaStream_t s, int sms) {
 
 template <int FMT>
 cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
-    // few rows: the swapped (weight-streaming) form
-    if (p.M <= 16) return launch_decode_nt<FMT, 16>(p, s, sms);
-    if (p.M <= 32) return launch_decode_nt<FMT, 32>(p, s, sms);
-    if (p.M <= 64) return launch_decode_nt<FMT, 64>(p, s, sms);
+    // few rows: the swapped (weight-streaming) form; the SwiGLU epilogue
+    // exists in the row-tiled form only
+    if (!p.swiglu) {
+        if (p.M <= 16) return launch_decode_nt<FMT, 16>(p, s, sms);
+        if (p.M <= 32) return launch_decode_nt<FMT, 32>(p, s, sms);
+        if (p.M <= 64) return launch_decode_nt<FMT, 64>(p, s, sms);
+    }
     Sched sc{};
     sc.mt_count = (int)((p.M + BM - 1) / BM);
     sc.nt_count = p.N / BN;

@@ -15,7 +15,11 @@
 // a norm, phase 1 is a plain maximum over the whole tensor, spread over every
 // lane.  Phases 2 and 3 spread (row, 256-element segment) items over every
 // warp.  MXFP4 has no tensor scale, so its backbone and residual are produced
-// in one pass (after the RMS barrier when there is a norm).
+// in one pass (after the RMS barrier when there is a norm).  When the
+// producer of X has already taken A_b = max |X| (a no-norm input, e.g. the
+// SwiGLU epilogue of the gate+up linear), phase 1 and its barrier are
+// skipped: with the shared residual scale the whole prepare is then one
+// barrier-free pass.
 //
 // Every floating-point step is one correctly rounded fp32 operation
 // (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn, no contraction), so the
@@ -52,6 +56,7 @@ struct PrepArgs {
     float* rs_tscale;
     uint8_t* mask;           // optional
     uint32_t* ws;            // [0] amax_b bits, [1] amax_r bits, [2] barrier, then rinv[M], mu[M]
+    const float* amax_in;    // GIVEN: A_b = max |X| from the producer
 };
 
 __device__ __forceinline__ float* ws_rinv(uint32_t* ws) {
@@ -317,14 +322,16 @@ struct LaneBlock {
 // once (keep-all, no norm, no residual).  NM24: the 2-of-4 mask.  RS: the
 // residual takes the backbone's tensor scale (NVFP4), so it is finished in
 // phase 2 with the backbone's reciprocal table and phase 3 does not exist.
+// GIVEN: no norm, A_b read from a.amax_in, no phase 1.
 // ------------------------------------------------------------------------
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS, bool LN>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS, bool LN, bool GIVEN>
 __global__ void __launch_bounds__(kThreads, 2)
 prepare_kernel(PrepArgs a) {
     __shared__ float s_inv[128];
     __shared__ float s_red[kWarps];
     using LB = LaneBlock<FMT, HAS_GAMMA, LN>;
     static_assert(!LN || HAS_GAMMA, "LayerNorm takes gamma");
+    static_assert(!GIVEN || (FMT == 0 && !HAS_GAMMA && !WEIGHT), "a given amax: NVFP4, no norm");
     const bool has_beta = LN && a.beta != nullptr;
     constexpr int E = LB::E;
 
@@ -341,7 +348,7 @@ prepare_kernel(PrepArgs a) {
 
     // ---------------- phase 1: rinv per row, A_b = max |y| ----------------
     float amax = 0.0f;
-    if (FMT == 0 && !HAS_GAMMA) {
+    if (FMT == 0 && !HAS_GAMMA && !GIVEN) {
         // y = x, and A_b = max |x| needs no row structure: lane i of the
         // grid reads chunks i, i + L, ..., i + 15L (L = lanes in the grid),
         // sixteen loads in flight, then the next 16L chunks.  The magnitude
@@ -447,7 +454,7 @@ prepare_kernel(PrepArgs a) {
         }
     }
 
-    if (FMT == 0) {
+    if (FMT == 0 && !GIVEN) {
         block_amax_to_global(amax, &a.ws[0], s_red);
         grid_barrier(&a.ws[2], gridDim.x);
     } else if (HAS_GAMMA) {
@@ -457,7 +464,7 @@ prepare_kernel(PrepArgs a) {
     // ------- phase 2: mask, backbone, residual amax (and MXFP4 residual) -------
     NvScale sb{1.0f, 1.0f, 1.0f};
     if (FMT == 0) {
-        sb = nv_scale(__uint_as_float(ld_acquire_gpu(&a.ws[0])));
+        sb = nv_scale(GIVEN ? *a.amax_in : __uint_as_float(ld_acquire_gpu(&a.ws[0])));
         fill_inv_table(s_inv, sb.genc);
         if (blockIdx.x == 0 && threadIdx.x == 0) {
             *a.bb_tscale = sb.gdec;
@@ -582,7 +589,7 @@ prepare_kernel(PrepArgs a) {
     if (FMT == 1 || WEIGHT || RS) return;
 
     block_amax_to_global(ramax, &a.ws[1], s_red);
-    grid_barrier(&a.ws[2], 2u * gridDim.x);
+    grid_barrier(&a.ws[2], (GIVEN ? 1u : 2u) * gridDim.x);   // counts on from phase 1's
 
     // ---------------- phase 3: residual codes with G_r ----------------
     NvScale sr = nv_scale(__uint_as_float(ld_acquire_gpu(&a.ws[1])));
@@ -642,9 +649,10 @@ prepare_kernel(PrepArgs a) {
     }
 }
 
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false, bool LN = false>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false, bool LN = false,
+          bool GIVEN = false>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
-    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN>;
+    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN, GIVEN>;
     // same for every device of one architecture; a repeated query is harmless
     static std::atomic<int> cached{0};
     int blocks_per_sm = cached.load(std::memory_order_relaxed);
@@ -669,17 +677,20 @@ cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     attr[0].id = cudaLaunchAttributeCooperative;   // grid barriers: all blocks co-resident
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = (FMT == 0 || HAS_GAMMA) ? 1 : 0;   // any grid barrier needs co-residency
+    // any grid barrier needs co-residency: after phase 1 (a norm, or an NVFP4
+    // amax taken here) or before phase 3 (NVFP4 with its own residual scale)
+    const bool barrier = HAS_GAMMA || (FMT == 0 && !GIVEN) || (FMT == 0 && !WEIGHT && !RS);
+    cfg.numAttrs = barrier ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kfn, a);
 }
 
-template <int FMT, bool HAS_GAMMA, bool WEIGHT, bool RS = false, bool LN = false>
+template <int FMT, bool HAS_GAMMA, bool WEIGHT, bool RS = false, bool LN = false, bool GIVEN = false>
 cudaError_t launch_m(const PrepArgs& a, int m, cudaStream_t s, int sms) {
     switch (m) {
-        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false, RS, LN>(a, s, sms);
-        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true, RS, LN>(a, s, sms)
-                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false, RS, LN>(a, s, sms);
-        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false, RS, LN>(a, s, sms);
+        case 2: return launch_one<FMT, HAS_GAMMA, 2, WEIGHT, false, RS, LN, GIVEN>(a, s, sms);
+        case 4: return a.n == 2 ? launch_one<FMT, HAS_GAMMA, 4, WEIGHT, true, RS, LN, GIVEN>(a, s, sms)
+                                : launch_one<FMT, HAS_GAMMA, 4, WEIGHT, false, RS, LN, GIVEN>(a, s, sms);
+        default: return launch_one<FMT, HAS_GAMMA, 8, WEIGHT, false, RS, LN, GIVEN>(a, s, sms);
     }
 }
 
@@ -707,9 +718,16 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     a.rs_tscale = p.rs_tscale;
     a.mask = static_cast<uint8_t*>(p.mask);
     a.ws = static_cast<uint32_t*>(p.ws);
-    cudaError_t e = cudaMemsetAsync(p.ws, 0, 64, s);
-    if (e != cudaSuccess) return e;
+    a.amax_in = p.amax;
     const bool g = p.gamma != nullptr;
+    // the workspace header (maxima, barrier counter) starts at zero, unless
+    // the launch uses none of it: MXFP4 without a norm, or a given amax with
+    // the shared residual scale (one pass, no barrier)
+    const bool no_ws = (p.fmt == 1 && !g) || (p.fmt == 0 && p.amax && p.residual_shared && !p.weight);
+    if (!no_ws) {
+        cudaError_t e = cudaMemsetAsync(p.ws, 0, 64, s);
+        if (e != cudaSuccess) return e;
+    }
     if (p.weight) {
         return p.fmt == 0 ? launch_one<0, false, 8, true, false>(a, s, sms)
                           : launch_one<1, false, 8, true, false>(a, s, sms);
@@ -718,6 +736,10 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
         if (p.fmt == 1) return launch_m<1, true, false, false, true>(a, p.m, s, sms);
         return p.residual_shared ? launch_m<0, true, false, true, true>(a, p.m, s, sms)
                                  : launch_m<0, true, false, false, true>(a, p.m, s, sms);
+    }
+    if (p.fmt == 0 && p.amax) {   // no norm, A_b from the producer
+        return p.residual_shared ? launch_m<0, false, false, true, false, true>(a, p.m, s, sms)
+                                 : launch_m<0, false, false, false, false, true>(a, p.m, s, sms);
     }
     if (p.fmt == 0 && p.residual_shared)
         return g ? launch_m<0, true, false, true>(a, p.m, s, sms) : launch_m<0, false, false, true>(a, p.m, s, sms);

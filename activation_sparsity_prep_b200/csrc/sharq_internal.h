@@ -20,6 +20,7 @@ struct PrepareLaunch {
     int K, n, m, fmt;
     bool weight;          // quantise a whole weight tensor (keep-all, no residual)
     bool residual_shared; // NVFP4 residual quantised with the backbone's tensor scale
+    const float* amax;    // no-norm prepare with A_b = max |X| given by the producer, or null
     void* bb_codes;
     void* bb_scales;
     float* bb_tscale;
@@ -48,6 +49,8 @@ struct LinearLaunch {
     void* Y;
     int y_fp32;
     bool one_acc;             // G_b == G_r: both paths into one accumulator
+    bool swiglu;              // epilogue emits silu(gate) * up, [M, N/2] bf16, and max |H|
+    float* amax;              // swiglu: max |H| (device fp32)
     // grouped form
     const int32_t* row_index; // may be null
     const int32_t* offsets;   // null for the plain linear

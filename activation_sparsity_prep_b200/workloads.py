@@ -162,6 +162,13 @@ WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload(
         "tiny", 1, "normal_outlier",
         (Linear("tiny", 256, 256, True, 0),), Ms=(16,)),
+    # a small SwiGLU MLP (gate+up 256 -> 2 x 128, down 128 -> 256) for the
+    # producer-fused path's quick checks
+    "tiny_mlp": Workload(
+        "tiny_mlp", 7, "laplace_outlier",
+        (Linear("gate_up", 256, 512, True, 0),
+         Linear("down", 256, 256, False, 1)),
+        Ms=(16,)),
     "llama8b": Workload(
         "llama8b", 2, "laplace_outlier",
         (Linear("qkv", 4096, 6144, True, 0),

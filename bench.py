@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--nm", default="2:4", help="n:m of the backbone mask")
     ap.add_argument("--residual", choices=["own", "shared"], default="own",
                     help="tensor scale of the NVFP4 residual: its own (default) or the backbone's")
+    ap.add_argument("--fuse-mlp", action="store_true",
+                    help="SwiGLU MLP with the producer-fused prepare: gate+up writes silu(gate)*up "
+                         "and its amax, down prepares that H without its own amax pass")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -205,18 +208,39 @@ def profiled_traffic(launch_key: str, sha: str):
 
 # ------------------------------------------------------------ CPU arm ----
 
-def oracle_sample_step(linears, rows: int, quantized, fmt="nvfp4", n=2, m=4, residual="own"):
+def oracle_sample_step(linears, rows: int, quantized, fmt="nvfp4", n=2, m=4, residual="own",
+                       fuse_mlp=False):
     """One bounded oracle step: prepare and linear of the first `rows` rows
-    of every linear.  Returns (seconds, effective flops of the sample)."""
+    of every linear.  fuse_mlp: the down projection's input is the SwiGLU of
+    the gate+up output (rounded to bf16) instead of its synthetic tensor.
+    Returns (seconds, effective flops of the sample)."""
     import oracle
     t0 = time.perf_counter()
     fl = 0.0
+    H = None
     for (L, d), Wq in zip(linears, quantized):
-        P = oracle.prepare(d["X"][:rows], d["gamma"], wl.EPS, n, m, fmt, residual_scale=residual,
+        X = d["X"][:rows] if not (fuse_mlp and L.name == "down") else H
+        P = oracle.prepare(X, d["gamma"], wl.EPS, n, m, fmt, residual_scale=residual,
                            norm=d["norm"], beta=d["beta"])
-        oracle.linear(P, Wq)
+        if fuse_mlp and L.name == "gate_up":
+            H = oracle.bf16_rne_from_f64(oracle.swiglu_linear(P, Wq))
+        else:
+            oracle.linear(P, Wq)
         fl += 2.0 * rows * L.N * L.K
     return time.perf_counter() - t0, fl
+
+
+def mlp_fusable(W) -> bool:
+    names = [L.name for L in W.linears]
+    return W.moe is None and "gate_up" in names and "down" in names
+
+
+def gate_up_interleaved(W_bits):
+    """The synthetic gate+up weight [2I, K] read as gate rows then up rows,
+    in the fused linear's interleaved layout."""
+    import oracle
+    I = W_bits.shape[0] // 2
+    return oracle.interleave_gate_up(W_bits[:I], W_bits[I:])
 
 
 def oracle_moe_sample_step(W, sample, fmt="nvfp4", n=2, m=4, residual="own"):
@@ -272,18 +296,21 @@ def blas_threads():
 def cpu_baseline(linears, args, budget_s: float = 15.0, rows: int = 16):
     import oracle
     n_, m_ = nm_of(args)
-    quantized = [oracle.quantize_weight(d["W"], args.fmt) for _, d in linears]
+    quantized = [oracle.quantize_weight(gate_up_interleaved(d["W"]) if args.fuse_mlp and L.name == "gate_up"
+                                        else d["W"], args.fmt) for L, d in linears]
     total_t, total_f, n = 0.0, 0.0, 0
     while total_t < budget_s and n < 50:
-        t, f = oracle_sample_step(linears, rows, quantized, args.fmt, n_, m_, args.residual)
+        t, f = oracle_sample_step(linears, rows, quantized, args.fmt, n_, m_, args.residual,
+                                  args.fuse_mlp)
         total_t += t
         total_f += f
         n += 1
     return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
             "kind": "oracle",
             "sample": f"{n} passes of: oracle prepare + fp64 two-path linear on the first {rows} "
-                      f"rows of each of the {len(linears)} linears (all N); prepare single-threaded C, "
-                      f"GEMM numpy/OpenBLAS fp64"}
+                      f"rows of each of the {len(linears)} linears (all N"
+                      f"{'; SwiGLU of gate+up feeds down' if args.fuse_mlp else ''}); prepare "
+                      f"single-threaded C, GEMM numpy/OpenBLAS fp64"}
 
 
 def workload_desc(W, M):
@@ -300,6 +327,9 @@ def workload_desc(W, M):
 def bench_config(args, W, M):
     return {"workload": workload_desc(W, M), "M": M, "fmt": args.fmt, "nm": args.nm,
             "residual_scale": args.residual,
+            "mlp": ("producer-fused: gate_up writes H = silu(gate)*up and max|H| (SwiGLU epilogue), "
+                    "down prepares that H from the producer's amax" if args.fuse_mlp else
+                    "separate: every linear reads its own synthetic input"),
             "l2": "flushed between timed steps (512 MiB write)",
             "timing": "CUDA graph per step, per-kernel external events"}
 
@@ -314,10 +344,13 @@ def run_reference(args):
     if W.moe is None:
         linears = make_inputs(W, args.M)
         import oracle
-        quantized = [oracle.quantize_weight(d["W"], args.fmt) for _, d in linears]
+        quantized = [oracle.quantize_weight(gate_up_interleaved(d["W"]) if args.fuse_mlp and L.name == "gate_up"
+                                            else d["W"], args.fmt) for L, d in linears]
         rows = 16
-        step = lambda: oracle_sample_step(linears, rows, quantized, args.fmt, n, m, args.residual)
-        what = f"first {rows} rows of each linear per step (all N), of M={args.M}"
+        step = lambda: oracle_sample_step(linears, rows, quantized, args.fmt, n, m, args.residual,
+                                          args.fuse_mlp)
+        what = (f"first {rows} rows of each linear per step (all N), of M={args.M}"
+                + ("; the SwiGLU of gate+up (bf16) feeds down" if args.fuse_mlp else ""))
         M = args.M
     else:
         sample = moe_reference_sample(W, args.fmt)
@@ -371,23 +404,44 @@ def build_units(args, dev):
     units = []
     if W.moe is None:
         M = args.M
+        fused = None          # (H, amax) of the SwiGLU gate+up, when the MLP is fused
         for L in W.linears:
             d = wl.linear_inputs(W, L, M)
-            X, g = up(d["X"]), (None if d["gamma"] is None else up(d["gamma"]))
+            g = None if d["gamma"] is None else up(d["gamma"])
             b = None if d["beta"] is None else up(d["beta"])
+            swiglu = args.fuse_mlp and L.name == "gate_up"
             Wt = up(d["W"])
+            if swiglu:
+                Wt = sq.interleave_gate_up(Wt[:L.N // 2], Wt[L.N // 2:])
             w = sq.quantize_weight(Wt, fmt)
             del Wt
             P = sq.Prepared.empty(M, L.K, n, m, fmt, device=dev, residual_scale=args.residual)
             ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
-            Y = torch.empty((M, L.N), dtype=bf, device=dev)
-            u = dict(name=L.name, rows=M, prep_rows=M, N=L.N, K=L.K, X=X, Y=Y)
+            if swiglu:
+                Y = torch.empty((M, L.N // 2), dtype=bf, device=dev)
+                amax = torch.empty((1,), dtype=torch.float32, device=dev)
+                fused = (Y, amax)
+            else:
+                Y = torch.empty((M, L.N), dtype=bf, device=dev)
+            if args.fuse_mlp and L.name == "down":
+                X, amax = fused
+                u = dict(name=L.name, rows=M, prep_rows=M, N=L.N, K=L.K, X=X, Y=Y, host_input=False)
+                u["prep"] = (lambda X=X, amax=amax, P=P, ws=ws:
+                             sq.prepare_amax(X, amax, n, m, fmt, out=P, ws=ws))
+                u["gemm"] = (lambda P=P, w=w, Y=Y: sq.linear(P, w, out=Y))
+                units.append(u)
+                continue
+            X = up(d["X"])
+            u = dict(name=L.name, rows=M, prep_rows=M, N=L.N, K=L.K, X=X, Y=Y, swiglu=swiglu)
+            if swiglu:
+                u["gemm"] = (lambda P=P, w=w, Y=Y, amax=amax: sq.linear_swiglu(P, w, out=Y, amax=amax))
             if L.layernorm:
                 u["prep"] = (lambda X=X, g=g, b=b, P=P, ws=ws:
                              sq.prepare_layernorm(X, g, b, wl.EPS, n, m, fmt, out=P, ws=ws))
             else:
                 u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
-            u["gemm"] = (lambda P=P, w=w, Y=Y: sq.linear(P, w, out=Y))
+            if "gemm" not in u:
+                u["gemm"] = (lambda P=P, w=w, Y=Y: sq.linear(P, w, out=Y))
             units.append(u)
         return units, M
     T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
@@ -503,14 +557,14 @@ def run_sharq(args):
     # + scales once, activation codes + scales of both paths, bf16 output
     sfb = 1.0 / (16 if fmt == 0 else 32)
     lin_bytes = (ud["N"] * ud["K"] * (0.5 + sfb) + ud["rows"] * ud["K"] * 2 * (0.5 + sfb)
-                 + 2.0 * ud["rows"] * ud["N"])
+                 + 2.0 * ud["Y"].numel())
     lin_flops = alg_factor * ud["rows"] * ud["N"] * ud["K"]
     hbm_bound = lin_bytes / (hbm * 1e9) > lin_flops / (fp4_peak * 1e12)
     if hbm_bound:
         achieved, lin_peak, lin_unit = lin_bytes / lin_t[dom] / 1e9, hbm, "GB/s"
     else:
         achieved, lin_peak, lin_unit = lin_flops / lin_t[dom] / 1e12, fp4_peak, "TFLOP/s"
-    lin_key = f"linear_{args.fmt}_{args.workload}_{ud['name']}_M{args.M}"
+    lin_key = f"linear_{args.fmt}_{args.workload}_{ud['name']}{'_swiglu' if ud.get('swiglu') else ''}_M{args.M}"
     traffic = profiled_traffic(lin_key, source_sha("linear.cu", "common.cuh"))
     # Prepare roofline on its largest launch (algorithmic bytes per element:
     # read X 2, backbone codes 0.5 (zero-filled) + scales, residual codes 0.5 + scales)
@@ -524,7 +578,8 @@ def run_sharq(args):
     # end-to-end: host inputs (pinned) in, host outputs out, every step
     e2e = None
     if not args.no_e2e:
-        hx = [u["X"].cpu().pin_memory() for u in units]
+        fed = [u for u in units if u.get("host_input", True)]      # inputs that come from the host
+        hx = [u["X"].cpu().pin_memory() for u in fed]
         hy = [torch.empty(u["Y"].shape, dtype=u["Y"].dtype, pin_memory=True) for u in units]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ts = []
@@ -532,7 +587,7 @@ def run_sharq(args):
         for it in range(args.warmup + args.steps):
             flush.zero_()
             e0.record(cur)
-            for u, h in zip(units, hx):
+            for u, h in zip(fed, hx):
                 u["X"].copy_(h, non_blocking=True)
             g.replay()
             for u, h in zip(units, hy):
@@ -566,8 +621,8 @@ def run_sharq(args):
                          "traffic": traffic, "algorithmic_bytes": lin_bytes,
                          "algorithmic_flops": lin_flops,
                          "kernel": f"{'moe_' if wl.WORKLOADS[args.workload].moe else ''}linear_kernel "
-                                   f"(two-path FP4 GEMM), {ud['name']} launch rows={ud['rows']} "
-                                   f"N={ud['N']} K={ud['K']}",
+                                   f"(two-path FP4 GEMM{', SwiGLU epilogue' if ud.get('swiglu') else ''}), "
+                                   f"{ud['name']} launch rows={ud['rows']} N={ud['N']} K={ud['K']}",
                          "peak_note": (f"{src} copy bandwidth" if hbm_bound else
                                        f"dense FP4 = 4 x {src} bf16 burst ({bf16:.0f} TFLOP/s)"),
                          "achieved_note": f"{alg_factor:g}*M*N*K per launch ({n}:{m} backbone at 2x "
@@ -601,6 +656,8 @@ def main():
     if args.M is None:
         Ms = wl.WORKLOADS[args.workload].Ms
         args.M = 2048 if args.workload == "llama8b" else (Ms[0] if Ms else 0)
+    if args.fuse_mlp and not mlp_fusable(wl.WORKLOADS[args.workload]):
+        raise SystemExit("--fuse-mlp needs a dense workload with gate_up and down linears")
     if args.impl == "reference":
         return run_reference(args)
     return run_sharq(args)

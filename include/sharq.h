@@ -177,6 +177,40 @@ SHARQ_API sharq_status sharq_prepare_layernorm(const void* X_bf16, const void* g
 SHARQ_API sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w,
                           void* Y, int y_is_fp32, void* stream);
 
+/* Producer-fused MLP (the preparation operator of the Abstract, moved in
+ * front of the down projection's producer).  For a SwiGLU MLP the down
+ * projection's input is H = silu(x W_g^T) * (x W_u^T) (Shazeer, "GLU Variants
+ * Improve Transformer", 2020).  sharq_linear_swiglu runs the two-path linear
+ * of the gate+up projection and applies the gate in its epilogue:
+ *   w   holds 2I rows, interleaved per 128: rows 128t .. 128t+63 are gate
+ *       rows 64t .. 64t+63, rows 128t+64 .. 128t+127 the up rows with the
+ *       same indices (w->N = 2I, a multiple of 128);
+ *   g,u = the fp32 values sharq_linear would round to bf16 for those rows;
+ *   H[i, 64t+j] = bf16_rne(fl(silu(g) * u)), silu(g) = g / (1 + e^-g) in
+ *       fp32 with the fast exponential and divide: relative error within
+ *       (5 + 1.2 |g|) 2^-23 for g > -87 (0 below, where |silu| < 1e-36);
+ *       H is bf16 [M, I] (16-byte aligned, device);
+ *   *h_amax = max |H| over the whole tensor (fp32 holding a bf16 value;
+ *       device pointer, 4-byte aligned, written by this call; 0 for M = 0).
+ * The row-tiled kernel serves every M here (no decode form).  Errors as
+ * sharq_linear; NULL h_amax is SHARQ_ERR_INVALID_ARG. */
+SHARQ_API sharq_status sharq_linear_swiglu(const sharq_prepared* x, const sharq_weight* w, void* H,
+                                           float* h_amax, void* stream);
+
+/* The preparation operator for a no-norm input whose producer has already
+ * taken A = max |X| (sharq_linear_swiglu's h_amax): identical outputs to
+ * sharq_prepare(X, NULL, ...) whenever *amax == max |X|, without the pass
+ * that computes it.  The backbone's block maxima are those of X (the largest
+ * entry of every group is always kept), so A is also the backbone's amax.
+ * With SHARQ_RESIDUAL_SHARED the NVFP4 prepare is then a single pass without
+ * a grid barrier.  amax: device fp32, 4-byte aligned, not NULL; a value
+ * above max |X| is accepted (coarser scales), one below it saturates codes.
+ * MXFP4 has no tensor scale and does not read it.  Buffers, workspace and
+ * errors as sharq_prepare. */
+SHARQ_API sharq_status sharq_prepare_amax(const void* X_bf16, const float* amax,
+                                          const sharq_prepared* out, void* ws, size_t ws_bytes,
+                                          void* stream);
+
 /* Grouped (mixture-of-experts) form of sharq_linear (the pages evaluate the
  * method on a mixture-of-experts model; each expert is a SharQ linear):
  * dispatched row t (0 <= t < T) reads prepared row row_index[t] (row_index

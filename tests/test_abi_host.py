@@ -117,3 +117,44 @@ def test_workload_inputs_carry_the_norm_kind():
     assert d["norm"] == "layernorm" and d["beta"].shape == (5120,) and d["gamma"].shape == (5120,)
     d = wl.linear_inputs(W, W.linears[1], 4)
     assert d["norm"] == "rms" and d["gamma"] is None and d["beta"] is None
+
+
+def test_swiglu_linear_rejects_bad_arguments_on_host():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 0)
+    assert L.sharq_linear_swiglu(ctypes.byref(cp), ctypes.byref(w), 0x1000, None, None) == 1     # no amax
+    assert L.sharq_linear_swiglu(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0x1002, None) == 1   # misaligned amax
+    assert L.sharq_linear_swiglu(ctypes.byref(cp), ctypes.byref(w), 0x1008, 0x1000, None) == 1   # misaligned H
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 192, 256, 0)                                           # N % 128
+    assert L.sharq_linear_swiglu(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0x1000, None) == 1
+    cp = _fake_prepared(rs=2)
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 0)
+    assert L.sharq_linear_swiglu(ctypes.byref(cp), ctypes.byref(w), 0x1000, 0x1000, None) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(K=100), dict(m=3), dict(n=0), dict(fmt=7), dict(p=0x1001), dict(rs=2)])
+def test_prepare_amax_rejects_bad_arguments_on_host(kw):
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared(**kw)
+    assert L.sharq_prepare_amax(0x1000, 0x1000, ctypes.byref(cp), 0x1000, 1 << 20, None) == 1
+
+
+def test_prepare_amax_needs_an_aligned_amax():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    assert L.sharq_prepare_amax(0x1000, None, ctypes.byref(cp), 0x1000, 1 << 20, None) == 1
+    assert L.sharq_prepare_amax(0x1000, 0x1001, ctypes.byref(cp), 0x1000, 1 << 20, None) == 1
+    assert L.sharq_prepare_amax(0x1000, 0x1000, ctypes.byref(cp), 0x1000, 8, None) == 1          # workspace
+
+
+def test_interleave_helper_matches_the_oracle_layout():
+    import torch
+
+    import oracle
+    from activation_sparsity_prep_b200 import workloads as wl
+    Wg, Wu = wl.weight(5, 1, 192, 256), wl.weight(5, 2, 192, 256)
+    got = sq.interleave_gate_up(torch.from_numpy(Wg.view(np.int16)), torch.from_numpy(Wu.view(np.int16)))
+    assert np.array_equal(got.numpy().view(np.uint16), oracle.interleave_gate_up(Wg, Wu))
+    with pytest.raises(ValueError):
+        sq.interleave_gate_up(torch.zeros(96, 256), torch.zeros(96, 256))

@@ -40,3 +40,16 @@ def test_reference_arm_follows_format_and_residual_options():
     j = _run("--workload", "tiny", "--fmt", "mxfp4", "--nm", "1:4", "--residual", "shared")
     assert j["config"]["fmt"] == "mxfp4" and j["config"]["nm"] == "1:4"
     assert j["config"]["residual_scale"] == "shared"
+
+
+def test_reference_arm_runs_the_fused_mlp():
+    j = _run("--workload", "tiny_mlp", "--fuse-mlp")
+    assert j["config"]["mlp"].startswith("producer-fused") and j["value"] > 0
+    assert "SwiGLU" in j["cpu_baseline"]["sample"]
+
+
+def test_fused_mlp_needs_gate_up_and_down():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--fuse-mlp", "--steps", "1", "--warmup", "0"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode != 0 and "gate_up and down" in out.stderr
