@@ -98,6 +98,9 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_moe_linear.argtypes = [ctypes.POINTER(_Prepared), P, P, I, I64,
                                        ctypes.POINTER(_Weight), P, I, P, SZ, P]
         L.sharq_moe_linear.restype = I
+        L.sharq_moe_linear_swiglu.argtypes = [ctypes.POINTER(_Prepared), P, P, I, I64,
+                                              ctypes.POINTER(_Weight), P, P, P, SZ, P]
+        L.sharq_moe_linear_swiglu.restype = I
         L.sharq_prepare_noalloc.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P]
         L.sharq_prepare_noalloc.restype = I
         L.sharq_last_device_status.argtypes = [P]
@@ -362,6 +365,30 @@ def moe_linear(x: Prepared, row_index, offsets, w: Weight, out_fp32: bool = Fals
                               ctypes.byref(cw), Y.data_ptr(), 1 if out_fp32 else 0,
                               ws.data_ptr(), ws.numel(), _stream(stream)))
     return Y
+
+
+def moe_linear_swiglu(x: Prepared, row_index, offsets, w: Weight, out=None, amax=None, ws=None,
+                      T: Optional[int] = None, stream=None):
+    """Grouped gate+up linear with the SwiGLU epilogue over E stacked
+    interleaved expert weights: returns (H bf16 [T, w.N/2] in dispatch order,
+    amax fp32 [1] = max |H|)."""
+    import torch
+    L = load_sharq_ops()
+    if T is None:
+        T = int(row_index.numel()) if row_index is not None else x.M
+    E = int(offsets.numel()) - 1
+    dev = x.bb_scales.device
+    H = out if out is not None else torch.empty((T, w.N // 2), dtype=torch.bfloat16, device=dev)
+    a = amax if amax is not None else torch.empty((1,), dtype=torch.float32, device=dev)
+    need = moe_workspace_bytes(T, E, x.K, x.fmt)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=dev)
+    cx, cw = x._c(), w._c()
+    _check("sharq_moe_linear_swiglu",
+           L.sharq_moe_linear_swiglu(ctypes.byref(cx), _ptr(row_index), offsets.data_ptr(), E, T,
+                                     ctypes.byref(cw), H.data_ptr(), a.data_ptr(), ws.data_ptr(),
+                                     ws.numel(), _stream(stream)))
+    return H, a
 
 
 def last_device_status(stream=None) -> int:

@@ -190,10 +190,10 @@ size_t sharq_moe_workspace_bytes(int64_t T, int E, int K, int fmt) {
     return sharq::moe_ws_bytes(T, E, K, fmt);
 }
 
-sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
-                              const int32_t* expert_offsets, int E, int64_t T,
-                              const sharq_weight* w, void* Y, int y_is_fp32, void* ws,
-                              size_t ws_bytes, void* stream) {
+static sharq_status moe_common(const sharq_prepared* x, const int32_t* row_index,
+                               const int32_t* expert_offsets, int E, int64_t T, const sharq_weight* w,
+                               void* Y, int y_is_fp32, float* h_amax, void* ws, size_t ws_bytes,
+                               void* stream) {
     if (!x || !w) return SHARQ_ERR_INVALID_ARG;
     if (!expert_offsets || E <= 0 || T < 0 || (!row_index && T != x->M)) return SHARQ_ERR_INVALID_ARG;
     if (E > 256) return SHARQ_ERR_UNSUPPORTED;
@@ -209,10 +209,14 @@ sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
         return SHARQ_ERR_INVALID_ARG;
     if (!aligned16(x->bb_codes) || !aligned16(x->bb_scales) || !aligned16(x->rs_codes) ||
         !aligned16(x->rs_scales) || !aligned16(w->codes) || !aligned16(w->scales) || !aligned16(Y) ||
-        !aligned16(ws) || ((uintptr_t)row_index & 3u) || ((uintptr_t)expert_offsets & 3u))
+        !aligned16(ws) || ((uintptr_t)row_index & 3u) || ((uintptr_t)expert_offsets & 3u) ||
+        ((uintptr_t)h_amax & 3u))
         return SHARQ_ERR_INVALID_ARG;
     if (ws_bytes < sharq::moe_ws_bytes(T, E, x->K, x->fmt)) return SHARQ_ERR_INVALID_ARG;
-    if (T == 0) return SHARQ_OK;
+    if (T == 0) {
+        if (!h_amax) return SHARQ_OK;
+        return cuda_status(cudaMemsetAsync(h_amax, 0, sizeof(float), static_cast<cudaStream_t>(stream)));
+    }
     sharq::LinearLaunch p{};
     p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
     p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
@@ -220,8 +224,24 @@ sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
     p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
     p.one_acc = x->fmt == SHARQ_MXFP4 || x->residual_scale == SHARQ_RESIDUAL_SHARED;
     p.row_index = row_index; p.offsets = expert_offsets; p.E = E; p.T = T; p.ws = ws;
+    p.swiglu = h_amax != nullptr; p.amax = h_amax;
     return cuda_status(sharq::launch_moe_linear(p, static_cast<cudaStream_t>(stream),
                                                 sharq::device_sm_count()));
+}
+
+sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* row_index,
+                              const int32_t* expert_offsets, int E, int64_t T,
+                              const sharq_weight* w, void* Y, int y_is_fp32, void* ws,
+                              size_t ws_bytes, void* stream) {
+    return moe_common(x, row_index, expert_offsets, E, T, w, Y, y_is_fp32, nullptr, ws, ws_bytes, stream);
+}
+
+sharq_status sharq_moe_linear_swiglu(const sharq_prepared* x, const int32_t* row_index,
+                                     const int32_t* expert_offsets, int E, int64_t T,
+                                     const sharq_weight* w, void* H, float* h_amax, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    if (!h_amax) return SHARQ_ERR_INVALID_ARG;
+    return moe_common(x, row_index, expert_offsets, E, T, w, H, 0, h_amax, ws, ws_bytes, stream);
 }
 
 sharq_status sharq_last_device_status(void* stream) {

@@ -473,11 +473,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 // are not written.
                 const int64_t wrow0 = ti.y_row + q * 32;
                 __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(ep.Y);
-                if (!SW && sc.grouped) {
+                const int64_t ldy = SW ? ep.N / 2 : ep.N;     // H has N/2 columns
+                const int64_t ycol = SW ? col0 / 2 : col0;
+                if (sc.grouped) {
                     // 32 rows x 16 columns at a time: 16 rows x 32 bytes per store
                     uint8_t* stg = ssm->g.stage[q];
 #pragma unroll
-                    for (int hc = 0; hc < BN / 16; ++hc) {
+                    for (int hc = 0; hc < kOutCols / 16; ++hc) {
 #pragma unroll
                         for (int p = 0; p < 2; ++p)
                             *reinterpret_cast<uint4*>(stg + lane * 32 + 16 * (p ^ ((lane >> 2) & 1))) =
@@ -489,15 +491,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                             const int r = 16 * st + (lane >> 1), p = lane & 1;
                             const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 32 + 16 * (p ^ ((r >> 2) & 1)));
                             if (q * 32 + r < ti.rows)
-                                *reinterpret_cast<uint4*>(yb + (wrow0 + r) * ep.N + col0 + hc * 16 + p * 8) = v;
+                                *reinterpret_cast<uint4*>(yb + (wrow0 + r) * ldy + ycol + hc * 16 + p * 8) = v;
                         }
                         __syncwarp();
                     }
                 } else {
                     // 32 rows x 32 columns at a time: 8 rows x 64 bytes per store
                     uint8_t* stg = ssm->stage2[q];
-                    const int64_t ldy = SW ? ep.N / 2 : ep.N;     // H has N/2 columns
-                    const int64_t ycol = SW ? col0 / 2 : col0;
 #pragma unroll
                     for (int cc = 0; cc < kOutCols / 32; ++cc) {
 #pragma unroll

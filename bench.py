@@ -232,7 +232,7 @@ def oracle_sample_step(linears, rows: int, quantized, fmt="nvfp4", n=2, m=4, res
 
 def mlp_fusable(W) -> bool:
     names = [L.name for L in W.linears]
-    return W.moe is None and "gate_up" in names and "down" in names
+    return "gate_up" in names and "down" in names
 
 
 def gate_up_interleaved(W_bits):
@@ -243,25 +243,36 @@ def gate_up_interleaved(W_bits):
     return oracle.interleave_gate_up(W_bits[:I], W_bits[I:])
 
 
-def oracle_moe_sample_step(W, sample, fmt="nvfp4", n=2, m=4, residual="own"):
+def oracle_moe_sample_step(W, sample, fmt="nvfp4", n=2, m=4, residual="own", fuse_mlp=False):
     """Bounded oracle step of the grouped layer: every sampled dispatched row
-    through its own expert's two-path linear."""
+    through its own expert's two-path linear.  fuse_mlp: gate+up gives the
+    SwiGLU of each sampled (token, expert) row, which (rounded to bf16) is the
+    down projection's input for the same rows."""
     import oracle
     t0 = time.perf_counter()
     fl = 0.0
+    H = None
     for li, (L, X, g, rows, experts, wq) in enumerate(sample):
-        P = oracle.prepare(X, g, wl.EPS, n, m, fmt, residual_scale=residual)
+        P = oracle.prepare(X if X is not None else H, g, wl.EPS, n, m, fmt, residual_scale=residual)
+        Hs = np.zeros((len(rows), L.N // 2)) if fuse_mlp and li == 0 else None
         for e in sorted(set(experts.tolist())):
             sel = np.nonzero(experts == e)[0].astype(np.int32)
-            oracle.linear(oracle.gather_rows(P, rows[sel]), wq[e])
+            if Hs is not None:
+                Hs[sel] = oracle.swiglu_linear(oracle.gather_rows(P, rows[sel]), wq[e])
+            else:
+                oracle.linear(oracle.gather_rows(P, rows[sel]), wq[e])
             fl += 2.0 * len(sel) * L.N * L.K
+        if Hs is not None:
+            H = oracle.bf16_rne_from_f64(Hs)
     return time.perf_counter() - t0, fl
 
 
-def moe_reference_sample(W, fmt, tokens: int = 4):
+def moe_reference_sample(W, fmt, tokens: int = 4, fuse_mlp=False):
     """Sampled operands of the grouped layer: the first `tokens` tokens for
     gate+up (each with its top-k experts) and the first tokens*top-k
-    dispatched rows for down, with only the experts they reach quantised."""
+    dispatched rows for down, with only the experts they reach quantised.
+    fuse_mlp: down takes the same (token, expert) rows, its input the
+    gate+up SwiGLU (X None), and gate+up weights in the interleaved layout."""
     import oracle
     T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
     ex = wl.routing(W.cfg, T, E, topk)
@@ -272,14 +283,22 @@ def moe_reference_sample(W, fmt, tokens: int = 4):
             X = wl.activation(W.dist, W.cfg, L.index, tokens, L.K)
             rows = np.repeat(np.arange(tokens, dtype=np.int32), topk)
             experts = ex[:tokens].reshape(-1)
+        elif fuse_mlp:
+            X = None
+            rows = np.arange(tokens * topk, dtype=np.int32)
+            experts = ex[:tokens].reshape(-1)
         else:
             nrow = tokens * topk
             X = wl.activation(W.dist, W.cfg, L.index, T * topk, L.K)[:nrow]
             rows = np.arange(nrow, dtype=np.int32)
             experts = (np.searchsorted(off, rows, side="right") - 1).astype(np.int64)
         g = wl.gamma_ones(L.K) if L.norm else None
-        wq = {int(e): oracle.quantize_weight(wl.weight(W.cfg * 1000 + li, 100 + int(e), L.N, L.K), fmt)
-              for e in set(experts.tolist())}
+
+        def wbits(e, li=li, L=L):
+            Wb = wl.weight(W.cfg * 1000 + li, 100 + int(e), L.N, L.K)
+            return gate_up_interleaved(Wb) if fuse_mlp and li == 0 else Wb
+
+        wq = {int(e): oracle.quantize_weight(wbits(e), fmt) for e in set(experts.tolist())}
         sample.append((L, X, g, rows, experts, wq))
     return sample
 
@@ -353,10 +372,11 @@ def run_reference(args):
                 + ("; the SwiGLU of gate+up (bf16) feeds down" if args.fuse_mlp else ""))
         M = args.M
     else:
-        sample = moe_reference_sample(W, args.fmt)
-        step = lambda: oracle_moe_sample_step(W, sample, args.fmt, n, m, args.residual)
-        what = ("4 tokens through gate+up (each with its top-8 experts) and the first 32 dispatched "
-                "rows through down, per step")
+        sample = moe_reference_sample(W, args.fmt, fuse_mlp=args.fuse_mlp)
+        step = lambda: oracle_moe_sample_step(W, sample, args.fmt, n, m, args.residual, args.fuse_mlp)
+        what = ("4 tokens through gate+up (each with its top-8 experts) and "
+                + ("the SwiGLU of those 32 (token, expert) rows through down" if args.fuse_mlp else
+                   "the first 32 dispatched rows through down") + ", per step")
         M = W.moe["T"]
     for _ in range(args.warmup):
         step()
@@ -448,25 +468,42 @@ def build_units(args, dev):
     ri, off = wl.group_by_expert(wl.routing(W.cfg, T, E, topk), E)
     ri_d = torch.from_numpy(ri).to(dev)
     off_d = torch.from_numpy(off).to(dev)
+    fused = None
     for li, L in enumerate(W.linears):
         rows_in = T if li == 0 else T * topk             # gate_up reads tokens, down dispatched rows
-        X = up(wl.activation(W.dist, W.cfg, L.index, rows_in, L.K))
+        swiglu = args.fuse_mlp and li == 0
         g = up(wl.gamma_ones(L.K)) if L.norm else None
         w = sq.Weight.empty(L.N, L.K, fmt, device=dev, E=E)
         sb = sq.scale_bytes(L.N, L.K, fmt)
         for e in range(E):
             we = sq.Weight(w.codes[e], w.scales[e * sb:(e + 1) * sb], w.tensor_scale[e:e + 1],
                            L.N, L.K, w.fmt)
-            sq.quantize_weight(up(wl.weight(W.cfg * 1000 + li, 100 + e, L.N, L.K)), fmt, out=we)
+            Wt = up(wl.weight(W.cfg * 1000 + li, 100 + e, L.N, L.K))
+            if swiglu:
+                Wt = sq.interleave_gate_up(Wt[:L.N // 2], Wt[L.N // 2:])
+            sq.quantize_weight(Wt, fmt, out=we)
         P = sq.Prepared.empty(rows_in, L.K, n, m, fmt, device=dev, residual_scale=args.residual)
         ws = torch.empty(max(256, sq.prepare_workspace_bytes(rows_in, L.K, fmt)), dtype=torch.uint8, device=dev)
         mws = torch.empty(sq.moe_workspace_bytes(T * topk, E, L.K, fmt), dtype=torch.uint8, device=dev)
-        Y = torch.empty((T * topk, L.N), dtype=bf, device=dev)
+        Y = torch.empty((T * topk, L.N // 2 if swiglu else L.N), dtype=bf, device=dev)
         rix = ri_d if li == 0 else None
-        u = dict(name=L.name, rows=T * topk, prep_rows=rows_in, N=L.N, K=L.K, X=X, Y=Y)
-        u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
-        u["gemm"] = (lambda P=P, w=w, Y=Y, rix=rix, mws=mws:
-                     sq.moe_linear(P, rix, off_d, w, out=Y, ws=mws, T=T * topk))
+        if args.fuse_mlp and li == 1:
+            X, amax = fused
+            u = dict(name=L.name, rows=T * topk, prep_rows=rows_in, N=L.N, K=L.K, X=X, Y=Y,
+                     host_input=False)
+            u["prep"] = (lambda X=X, amax=amax, P=P, ws=ws: sq.prepare_amax(X, amax, n, m, fmt, out=P, ws=ws))
+        else:
+            X = up(wl.activation(W.dist, W.cfg, L.index, rows_in, L.K))
+            u = dict(name=L.name, rows=T * topk, prep_rows=rows_in, N=L.N, K=L.K, X=X, Y=Y, swiglu=swiglu)
+            u["prep"] = (lambda X=X, g=g, P=P, ws=ws: sq.prepare(X, g, wl.EPS, n, m, fmt, out=P, ws=ws))
+        if swiglu:
+            amax = torch.empty((1,), dtype=torch.float32, device=dev)
+            fused = (Y, amax)
+            u["gemm"] = (lambda P=P, w=w, Y=Y, rix=rix, mws=mws, amax=amax:
+                         sq.moe_linear_swiglu(P, rix, off_d, w, out=Y, amax=amax, ws=mws, T=T * topk))
+        else:
+            u["gemm"] = (lambda P=P, w=w, Y=Y, rix=rix, mws=mws:
+                         sq.moe_linear(P, rix, off_d, w, out=Y, ws=mws, T=T * topk))
         units.append(u)
     return units, T
 
@@ -657,7 +694,7 @@ def main():
         Ms = wl.WORKLOADS[args.workload].Ms
         args.M = 2048 if args.workload == "llama8b" else (Ms[0] if Ms else 0)
     if args.fuse_mlp and not mlp_fusable(wl.WORKLOADS[args.workload]):
-        raise SystemExit("--fuse-mlp needs a dense workload with gate_up and down linears")
+        raise SystemExit("--fuse-mlp needs a workload with gate_up and down linears")
     if args.impl == "reference":
         return run_reference(args)
     return run_sharq(args)

@@ -232,6 +232,19 @@ SHARQ_API sharq_status sharq_moe_linear(const sharq_prepared* x, const int32_t* 
                                         const sharq_weight* w, void* Y, int y_is_fp32,
                                         void* ws, size_t ws_bytes, void* stream);
 
+/* Grouped form of sharq_linear_swiglu (SwiGLU experts, e.g. the pages'
+ * mixture-of-experts model): every expert's gate+up weight is interleaved as
+ * for sharq_linear_swiglu (w holds E stacked [2I, K] weights, w->N = 2I), and
+ * row t of H is silu(gate) * up of dispatched row t through its own expert's
+ * weight, with the column pairing of sharq_linear_swiglu; H is bf16 [T, I]
+ * in dispatch order, the down projection's input in that order.
+ * *h_amax = max |H| over all T rows (0 for T = 0).  Arguments, workspace
+ * and errors as sharq_moe_linear; NULL h_amax is SHARQ_ERR_INVALID_ARG. */
+SHARQ_API sharq_status sharq_moe_linear_swiglu(const sharq_prepared* x, const int32_t* row_index,
+                                               const int32_t* expert_offsets, int E, int64_t T,
+                                               const sharq_weight* w, void* H, float* h_amax,
+                                               void* ws, size_t ws_bytes, void* stream);
+
 /* Largest M that sharq_prepare_noalloc() accepts (its fixed scratch array
  * holds 64 bytes plus 4 bytes per row: 1 MiB + 64 bytes in all). */
 #define SHARQ_NOALLOC_MAX_ROWS 262144

@@ -391,6 +391,30 @@ def swiglu_parts(prep: Prepared, w: Quantized, rows: Optional[np.ndarray] = None
     return g, u, ga, ua
 
 
+def moe_swiglu_parts(prep: Prepared, row_index: np.ndarray, offsets: np.ndarray, experts: list):
+    """Grouped form of swiglu_parts: (gate, up, |gate| bound, |up| bound) of
+    every dispatched row through its own expert's interleaved gate+up weight,
+    [T, I] each, in dispatch order."""
+    T = len(row_index)
+    grp = np.searchsorted(np.asarray(offsets), np.arange(T), side="right") - 1
+    I = experts[0].codes.shape[0] // 2
+    out = [np.zeros((T, I)) for _ in range(4)]
+    for e in np.unique(grp):
+        idx = np.nonzero(grp == e)[0]
+        parts = swiglu_parts(gather_rows(prep, np.asarray(row_index)[idx]), experts[int(e)])
+        for o, p in zip(out, parts):
+            o[idx] = p
+    return tuple(out)
+
+
+def moe_swiglu_linear(prep: Prepared, row_index: np.ndarray, offsets: np.ndarray,
+                      experts: list) -> np.ndarray:
+    """silu(gate) * up of every dispatched row through its own expert, fp64,
+    [T, I] in dispatch order."""
+    g, u, _, _ = moe_swiglu_parts(prep, row_index, offsets, experts)
+    return silu(g) * u
+
+
 def bf16_rne_from_f64(Y: np.ndarray) -> np.ndarray:
     """RNE(Y64) to bf16 bits, the reference for the bf16 output (fp64 -> bf16
     in one rounding, done exactly through the neighbouring bf16 values)."""

@@ -158,3 +158,16 @@ def test_interleave_helper_matches_the_oracle_layout():
     assert np.array_equal(got.numpy().view(np.uint16), oracle.interleave_gate_up(Wg, Wu))
     with pytest.raises(ValueError):
         sq.interleave_gate_up(torch.zeros(96, 256), torch.zeros(96, 256))
+
+
+def test_moe_swiglu_needs_an_amax():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    w = sq._Weight(0x1000, 0x1000, 0x1000, 256, 256, 0)
+    ws = sq.moe_workspace_bytes(16, 4, 256)
+    assert L.sharq_moe_linear_swiglu(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000,
+                                     None, 0x1000, ws, None) == 1
+    assert L.sharq_moe_linear_swiglu(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000,
+                                     0x1001, 0x1000, ws, None) == 1
+    assert L.sharq_moe_linear_swiglu(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000,
+                                     0x1000, 0x1000, ws - 1, None) == 1

@@ -53,3 +53,9 @@ def test_fused_mlp_needs_gate_up_and_down():
                           "--workload", "tiny", "--fuse-mlp", "--steps", "1", "--warmup", "0"],
                          capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert out.returncode != 0 and "gate_up and down" in out.stderr
+
+
+def test_reference_arm_runs_the_fused_moe_layer():
+    j = _run("--workload", "qwen3moe", "--fuse-mlp")
+    assert j["config"]["mlp"].startswith("producer-fused") and j["value"] > 0
+    assert "SwiGLU" in j["cpu_baseline"]["sample"]

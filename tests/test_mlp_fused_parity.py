@@ -31,11 +31,15 @@ def bf16_value(bits):
 
 def check_h(H, R, Rw, K, one_acc, rows=None):
     """H (device bf16) against the oracle's SwiGLU of the same operands."""
-    g, u, ga, ua = oracle.swiglu_parts(R, Rw, rows)
-    h = oracle.silu(g) * u
     got = to_np(H)
     if rows is not None:
         got = got[rows]
+    return check_h_parts(got, *oracle.swiglu_parts(R, Rw, rows), K, one_acc)
+
+
+def check_h_parts(got, g, u, ga, ua, K, one_acc):
+    """H bits against h = silu(g) u, with the bounds of g and u."""
+    h = oracle.silu(g) * u
     gamma = ((2 if one_acc else 1) * K / 64 + 2) * EPS23
     Eg, Eu = gamma * ga + 2.0 ** -126, gamma * ua + 2.0 ** -126
     s = np.abs(oracle.silu(g))
@@ -187,3 +191,89 @@ def test_fused_mlp_full_size_llama_prefill():
     R = oracle.prepare(d["X"], d["gamma"], wl.EPS, 2, 4, "nvfp4")
     rows = np.sort(np.random.default_rng(7).choice(M, 48, replace=False))
     check_h(H, R, oracle.quantize_weight(Wi, "nvfp4"), L.K, one_acc=False, rows=rows)
+
+
+def stacked_swiglu_weights(cfg, E, I, K, fmt):
+    Wis = [oracle.interleave_gate_up(wl.weight(cfg, 10 + e, I, K), wl.weight(cfg, 20 + e, I, K))
+           for e in range(E)]
+    w = sq.Weight.empty(2 * I, K, fmt, E=E)
+    sb = sq.scale_bytes(2 * I, K, fmt)
+    for e, Wi in enumerate(Wis):
+        we = sq.Weight(w.codes[e], w.scales[e * sb:(e + 1) * sb], w.tensor_scale[e:e + 1], 2 * I, K, w.fmt)
+        sq.quantize_weight(to_dev(Wi), fmt, out=we)
+    return Wis, w
+
+
+MOE_CASES = [
+    # tokens, experts, top-k, K, I, fmt, residual scale, routing
+    (200, 3, 2, 512, 128, "nvfp4", "own", "uniform"),
+    (70, 5, 2, 256, 64, "nvfp4", "own", "uneven"),       # experts 1, 2 (and most of 4) empty
+    (96, 4, 2, 256, 192, "mxfp4", "own", "uniform"),
+    (200, 3, 2, 512, 128, "nvfp4", "shared", "uniform"),
+]
+
+
+@pytest.mark.parametrize("T_tok,E,topk,K,I,fmt,rs,route", MOE_CASES)
+def test_moe_linear_swiglu_matches_oracle(T_tok, E, topk, K, I, fmt, rs, route):
+    X = wl.activation("laplace_outlier", 45, 0, T_tok, K)
+    g = wl.gamma_ones(K)
+    if route == "uneven":
+        ex = np.zeros((T_tok, 2), dtype=np.int32)
+        ex[:, 1] = 3
+        ex[:5, 1] = 4
+    else:
+        ex = wl.routing(45, T_tok, E, topk)
+    ri, off = wl.group_by_expert(ex.astype(np.int32), E)
+    Wis, w = stacked_swiglu_weights(45, E, I, K, fmt)
+    P = sq.prepare(to_dev(X), to_dev(g), wl.EPS, 2, 4, fmt, residual_scale=rs)
+    H, amax = sq.moe_linear_swiglu(P, torch.from_numpy(ri).cuda(), torch.from_numpy(off).cuda(), w)
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    assert H.shape == (len(ri), I)
+    R = oracle.prepare(X, g, wl.EPS, 2, 4, fmt, residual_scale=rs)
+    Rws = [oracle.quantize_weight(Wi, fmt) for Wi in Wis]
+    check_h_parts(to_np(H), *oracle.moe_swiglu_parts(R, ri, off, Rws), K,
+                  one_acc=fmt == "mxfp4" or rs == "shared")
+    check_amax(H, amax)
+
+
+def test_fused_moe_layer_full_size():
+    """The Qwen3-30B-A3B-shaped expert layer with the SwiGLU epilogue on the
+    grouped gate+up: H of 4 sampled experts against the oracle, the amax
+    over all 32768 dispatched rows, and the down prepare from that amax
+    bit-identical to the plain prepare of H."""
+    W = wl.WORKLOADS["qwen3moe"]
+    L = W.linears[0]
+    T, E, topk = W.moe["T"], W.moe["E"], W.moe["topk"]
+    I = L.N // 2
+    ri, off = wl.group_by_expert(wl.routing(W.cfg, T, E, topk), E)
+    X = wl.activation(W.dist, W.cfg, L.index, T, L.K)
+    g = wl.gamma_ones(L.K)
+    Wis = {}
+    w = sq.Weight.empty(L.N, L.K, "nvfp4", E=E)
+    sb = sq.scale_bytes(L.N, L.K, "nvfp4")
+    sampled = (0, 37, 64, 127)
+    for e in range(E):
+        Wb = wl.weight(W.cfg * 1000, 100 + e, L.N, L.K)
+        Wi = oracle.interleave_gate_up(Wb[:I], Wb[I:])
+        if e in sampled:
+            Wis[e] = Wi
+        we = sq.Weight(w.codes[e], w.scales[e * sb:(e + 1) * sb], w.tensor_scale[e:e + 1], L.N, L.K, w.fmt)
+        sq.quantize_weight(to_dev(Wi), "nvfp4", out=we)
+    P = sq.prepare(to_dev(X), to_dev(g), wl.EPS)
+    H, amax = sq.moe_linear_swiglu(P, torch.from_numpy(ri).cuda(), torch.from_numpy(off).cuda(), w)
+    Pd = sq.prepare_amax(H, amax)
+    Pref = sq.prepare(H, None)
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    check_amax(H, amax)
+    for f in ("bb_codes", "bb_scales", "bb_tscale", "rs_codes", "rs_scales", "rs_tscale"):
+        assert torch.equal(getattr(Pd, f), getattr(Pref, f)), f
+    R = oracle.prepare(X, g, wl.EPS)
+    got = to_np(H)
+    for e in sampled:
+        idx = np.arange(off[e], off[e + 1])
+        if len(idx) == 0:
+            continue
+        parts = oracle.swiglu_parts(oracle.gather_rows(R, ri[idx]), oracle.quantize_weight(Wis[e]))
+        check_h_parts(got[idx], *parts, L.K, one_acc=False)

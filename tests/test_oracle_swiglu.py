@@ -99,3 +99,20 @@ def test_swiglu_parts_bound_the_linear():
     g, u, ga, ua = oracle.swiglu_parts(P, Wq)
     assert np.all(ga >= np.abs(g)) and np.all(ua >= np.abs(u))
     np.testing.assert_array_equal(oracle.silu(g) * u, oracle.swiglu_linear(P, Wq))
+
+
+def test_moe_swiglu_is_the_per_expert_loop():
+    """The grouped oracle equals a loop of the plain SwiGLU linear over
+    dispatched rows, each through its own expert."""
+    T_tok, E, K, I = 12, 3, 256, 64
+    X = wl.activation("laplace_outlier", 93, 0, T_tok, K)
+    P = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4")
+    ex = wl.routing(93, T_tok, E, 2)
+    ri, off = wl.group_by_expert(ex.astype(np.int32), E)
+    Wq = [oracle.quantize_weight(oracle.interleave_gate_up(wl.weight(93, 10 + e, I, K),
+                                                           wl.weight(93, 20 + e, I, K))) for e in range(E)]
+    H = oracle.moe_swiglu_linear(P, ri, off, Wq)
+    for t in range(len(ri)):
+        e = int(np.searchsorted(off, t, side="right") - 1)
+        want = oracle.swiglu_linear(oracle.gather_rows(P, ri[t:t + 1]), Wq[e])[0]
+        np.testing.assert_array_equal(H[t], want)
