@@ -413,14 +413,17 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 constexpr int kOutCols = SW ? BN / 2 : BN;
                 uint32_t out[kOutCols / 2];
                 if constexpr (SW) {
-                    // columns j and 64 + j of the tile: gate and up of feature j.
-                    // Drain all 128 values first and hand the tensor memory back,
-                    // so the next tile's MMAs run under the SwiGLU arithmetic.
-                    float gv[BN / 2], uv[BN / 2];
+                    // columns j and 64 + j of the tile: gate and up of feature j,
+                    // 32 features at a time.  The tensor memory goes back after
+                    // the second drain, so the next tile's MMAs run under the
+                    // second half of the SwiGLU arithmetic; draining all 128
+                    // values first would spill registers (slower on both the
+                    // dense and the grouped launch).
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float gv[32], uv[32];
 #pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) {
+                        for (int half = 0; half < 2; ++half) {
                             uint32_t vb[32], vr[32];
                             const uint32_t c = half * (BN / 2) + cc * 32;
                             tmem_ld_32x32b_x32(src_b + lane_off + c, vb);
@@ -429,21 +432,23 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                             float* dst = half ? uv : gv;
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
-                                dst[cc * 32 + i] = ONE ? gb * __uint_as_float(vb[i])
-                                                       : gb * __uint_as_float(vb[i]) + gr * __uint_as_float(vr[i]);
+                                dst[i] = ONE ? gb * __uint_as_float(vb[i])
+                                             : gb * __uint_as_float(vb[i]) + gr * __uint_as_float(vr[i]);
                         }
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+                        if (cc == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+                        }
 #pragma unroll
-                    for (int h = 0; h < BN / 4; ++h) {
-                        const float h0 = __fmul_rn(silu_f32(gv[2 * h]), uv[2 * h]);
-                        const float h1 = __fmul_rn(silu_f32(gv[2 * h + 1]), uv[2 * h + 1]);
-                        __nv_bfloat162 p2 = __floats2bfloat162_rn(h0, h1);
-                        const uint32_t bits = *reinterpret_cast<uint32_t*>(&p2);
-                        out[h] = bits;
-                        if (row_ok) hmax = __vmaxu2(hmax, bits & 0x7FFF7FFFu);
+                        for (int h = 0; h < 16; ++h) {
+                            const float h0 = __fmul_rn(silu_f32(gv[2 * h]), uv[2 * h]);
+                            const float h1 = __fmul_rn(silu_f32(gv[2 * h + 1]), uv[2 * h + 1]);
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(h0, h1);
+                            const uint32_t bits = *reinterpret_cast<uint32_t*>(&p2);
+                            out[cc * 16 + h] = bits;
+                            if (row_ok) hmax = __vmaxu2(hmax, bits & 0x7FFF7FFFu);
+                        }
                     }
                 } else {
 #pragma unroll
