@@ -8,7 +8,10 @@ fallback: without the compiled library every call raises.
 SharQ paper, Abstract: a fused preparation operator (normalisation, an
 input-adaptive N:M mask, an FP4 backbone and an FP4 residual taken against
 the dequantised backbone) feeds a sparse FP4 GEMM and a dense FP4 GEMM that
-share one FP4 weight payload.
+share one FP4 weight payload.  For a SwiGLU MLP the gate+up linear can apply
+the gate in its epilogue (linear_swiglu / moe_linear_swiglu) and hand max |H|
+to the down projection's prepare (prepare_amax), which then skips its own
+amax pass.
 """
 from __future__ import annotations
 
@@ -21,8 +24,9 @@ from typing import Optional
 __all__ = [
     "NVFP4", "MXFP4", "SharqError", "load_sharq_ops", "scale_bytes",
     "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
-    "prepare", "prepare_noalloc", "linear", "moe_linear", "moe_workspace_bytes",
-    "last_device_status",
+    "prepare", "prepare_layernorm", "prepare_amax", "prepare_noalloc", "linear",
+    "linear_swiglu", "interleave_gate_up", "moe_linear", "moe_linear_swiglu",
+    "moe_workspace_bytes", "last_device_status",
 ]
 
 NVFP4, MXFP4 = 0, 1

@@ -14,6 +14,10 @@ FP4 linear) and of the prepare kernel, the CPU oracle baseline, the SM
 clocks seen during the timed region and an end-to-end figure with host
 buffers.  ``--impl reference`` times the CPU oracle instead.
 
+``--fuse-mlp`` runs the MLP producer-fused: the gate+up linear writes
+H = silu(gate) * up and max |H| in its epilogue, and the down projection
+prepares that H from the producer's amax instead of a synthetic input.
+
 Multi-GPU: the path has no exchange step at this scale; each rank runs an
 independent replica (weak scaling) and the slowest rank's time counts.
 """

@@ -171,3 +171,8 @@ def test_moe_swiglu_needs_an_amax():
                                      0x1001, 0x1000, ws, None) == 1
     assert L.sharq_moe_linear_swiglu(ctypes.byref(cp), None, 0x1000, 4, 16, ctypes.byref(w), 0x1000,
                                      0x1000, 0x1000, ws - 1, None) == 1
+
+
+def test_public_api_names_resolve():
+    for n in sq.__all__:
+        assert hasattr(sq, n), n
