@@ -1,0 +1,166 @@
+"""Pins of the oracle's fp32 normalisation arithmetic against an exact model
+of IEEE-754 binary32: every operation is carried out on exact rationals and
+rounded to nearest-even, written here from the definition of the format (24
+significant bits, normal exponents down to -126, subnormals below), with no
+use of the oracle's C code or of the CPU's fp32 unit.  Together with the
+fixed reduction order (32 lanes, chunk c to lane c mod 32, element order in
+a lane, xor butterfly 16..1) this fixes the RMSNorm and LayerNorm statistics
+bit for bit, so a compiler that contracted, reordered or widened any step of
+the oracle would fail here."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from activation_sparsity_prep_b200 import workloads as wl
+
+TWO = Fraction(2)
+
+
+def rne32(q: Fraction) -> Fraction:
+    """The binary32 value nearest to q, ties to the even significand."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()      # 2^e <= a < 2^(e+2)
+    if TWO ** e > a:
+        e -= 1
+    if TWO ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)                                               # subnormal spacing below
+    ulp = TWO ** (e - 23)
+    t = a / ulp
+    n = t.numerator // t.denominator
+    rem = t - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    assert n * ulp < TWO ** 128, "overflow is outside these pins"
+    return sign * n * ulp
+
+
+def f32_neighbours(v: Fraction):
+    f = np.float32(float(v))
+    assert Fraction(float(f)) == v
+    lo = np.nextafter(f, np.float32(-np.inf), dtype=np.float32)
+    hi = np.nextafter(f, np.float32(np.inf), dtype=np.float32)
+    return Fraction(float(lo)), Fraction(float(hi))
+
+
+def sqrt32(q: Fraction) -> Fraction:
+    """Correctly rounded binary32 square root of q >= 0: the candidate from
+    a double sqrt, moved until q lies between the squared midpoints to its
+    neighbours (ties to even)."""
+    assert q >= 0
+    if q == 0:
+        return Fraction(0)
+    c = rne32(Fraction(float(np.sqrt(float(q)))))
+    for _ in range(4):
+        lo, hi = f32_neighbours(c)
+        m_lo, m_hi = (lo + c) / 2, (c + hi) / 2
+        if m_lo * m_lo > q:
+            c = lo
+        elif m_hi * m_hi < q:
+            c = hi
+        else:
+            even = (int(np.float32(float(c)).view(np.uint32)) & 1) == 0
+            if m_hi * m_hi == q and not even:
+                c = hi
+            elif m_lo * m_lo == q and not even:
+                c = lo
+            return c
+    raise AssertionError("sqrt candidate did not settle")
+
+
+def bf16(b) -> Fraction:
+    return Fraction(float((np.uint32(b) << np.uint32(16)).view(np.float32)))
+
+
+def f32(v) -> Fraction:
+    return Fraction(float(np.float32(v)))
+
+
+def canonical_sum(vals):
+    lane = [Fraction(0)] * 32
+    for c in range(len(vals) // 8):
+        for t in range(8):
+            lane[c % 32] = rne32(lane[c % 32] + vals[8 * c + t])
+    o = 16
+    while o >= 1:
+        lane = [rne32(lane[l] + lane[l ^ o]) for l in range(32)]
+        o >>= 1
+    assert len(set(lane)) == 1          # every lane holds the same sum
+    return lane[0]
+
+
+def model_rinv(xb, eps):
+    x = [bf16(b) for b in xb]
+    S = canonical_sum([rne32(v * v) for v in x])
+    ms = rne32(S / len(x))
+    return rne32(1 / sqrt32(rne32(ms + f32(eps))))
+
+
+def model_ln(xb, eps):
+    x = [bf16(b) for b in xb]
+    mu = rne32(canonical_sum(x) / len(x))
+    d = [rne32(v - mu) for v in x]
+    var = rne32(canonical_sum([rne32(v * v) for v in d]) / len(x))
+    return mu, rne32(1 / sqrt32(rne32(var + f32(eps))))
+
+
+ROWS = [("laplace_outlier", 256), ("student_t", 512), ("normal_outlier", 1024), ("laplace_outlier", 768)]
+
+
+def test_model_rounding_against_known_values():
+    # the model itself, on values whose rounding is known by hand
+    assert rne32(Fraction(1) + TWO ** -24) == 1                       # tie: even (1.0)
+    assert rne32(Fraction(1) + 3 * TWO ** -24) == 1 + TWO ** -22      # tie: up to even
+    assert rne32(Fraction(1, 3)) == Fraction(float(np.float32(1 / 3)))
+    assert rne32(TWO ** -149 * Fraction(3, 2)) == TWO ** -148         # subnormal tie to even
+    assert sqrt32(Fraction(2)) == Fraction(float(np.float32(np.sqrt(np.float32(2)))))
+    assert sqrt32(Fraction(9, 4)) == Fraction(3, 2)
+
+
+@pytest.mark.parametrize("dist,K", ROWS)
+def test_rms_rinv_is_the_exact_fp32_model(dist, K):
+    X = wl.activation(dist, 95, K, 3, K)
+    for row in X:
+        got = Fraction(float(oracle.rms_rinv(row, 1e-6)))
+        assert got == model_rinv(row, 1e-6)
+
+
+@pytest.mark.parametrize("dist,K", ROWS)
+def test_layernorm_stats_are_the_exact_fp32_model(dist, K):
+    X = wl.activation(dist, 96, K, 2, K)
+    for row in X:
+        mu, rstd = oracle.ln_stats(row, 1e-6)
+        wmu, wrstd = model_ln(row, 1e-6)
+        assert Fraction(float(mu)) == wmu and Fraction(float(rstd)) == wrstd
+
+
+def test_rmsnorm_outputs_are_the_exact_fp32_model():
+    K = 256
+    X = wl.activation("laplace_outlier", 97, 0, 2, K)
+    g = wl.gamma_random(97, 0, K)
+    y = oracle.normalize(X, g, 1e-6)
+    for i, row in enumerate(X):
+        r = model_rinv(row, 1e-6)
+        want = [rne32(rne32(bf16(x) * r) * bf16(gk)) for x, gk in zip(row, g)]
+        assert [Fraction(float(v)) for v in y[i]] == want
+
+
+def test_the_model_sees_a_different_order():
+    """A plain left-to-right sum (a plausible mistake) gives other bits than
+    the oracle on at least one of these rows, so the pins above constrain
+    the order and not only the values."""
+    differs = False
+    for dist, K in ROWS:
+        for row in wl.activation(dist, 95, K, 3, K):
+            x = [bf16(b) for b in row]
+            S = Fraction(0)
+            for v in x:
+                S = rne32(S + rne32(v * v))
+            seq = rne32(1 / sqrt32(rne32(rne32(S / K) + f32(1e-6))))
+            differs |= seq != Fraction(float(oracle.rms_rinv(row, 1e-6)))
+    assert differs
