@@ -164,3 +164,120 @@ def test_the_model_sees_a_different_order():
             seq = rne32(1 / sqrt32(rne32(rne32(S / K) + f32(1e-6))))
             differs |= seq != Fraction(float(oracle.rms_rinv(row, 1e-6)))
     assert differs
+
+
+# ------------------------------------------------ the NVFP4 / MXFP4 chains --
+# The FP4 grids, written from the formats: E2M1 magnitudes of codes 0..7 and
+# E4M3 (bias 7, 3 mantissa bits, subnormal spacing 2^-9, largest 448).
+
+E2M1 = [Fraction(v) for v in ("0", "1/2", "1", "3/2", "2", "3", "4", "6")]
+E4M3 = ([Fraction(m, 8) * TWO ** -6 for m in range(8)]
+        + [(1 + Fraction(m, 8)) * TWO ** (e - 7) for e in range(1, 16) for m in range(8)])[:127]
+
+
+def nearest_even(grid, v: Fraction) -> int:
+    """Index (= code) of the grid value nearest to v >= 0, ties to the even
+    code, values past the top saturating."""
+    if v >= grid[-1]:
+        return len(grid) - 1
+    best = min(range(len(grid)), key=lambda c: (abs(grid[c] - v), c & 1))
+    return best
+
+
+def e2m1_code(v: Fraction, negative: bool) -> int:
+    return nearest_even(E2M1, abs(v)) | (8 if negative else 0)
+
+
+def keep_top2(vals):
+    order = sorted(range(4), key=lambda i: (-abs(vals[i]), i))
+    return {order[0], order[1]}
+
+
+def model_nvfp4(Y, A):
+    """Codes, block-scale codes and decode scale of Y (rows of exact values,
+    already masked) under the reading: G_enc = fl(2688 / A), k1 = fl(G_enc /
+    6), block code = E4M3(fl(amax_block * k1)), inv = fl(G_enc / e4m3(code)),
+    element code = E2M1(fl(y * inv)), G_dec = fl(A / 2688)."""
+    genc = rne32(Fraction(2688) / A) if A else Fraction(1)
+    gdec = rne32(A / Fraction(2688)) if A else Fraction(1)
+    k1 = rne32(genc / 6)
+    codes, scales = [], []
+    for row in Y:
+        rc, rs = [], []
+        for b0 in range(0, len(row), 16):
+            blk = row[b0:b0 + 16]
+            e = nearest_even(E4M3, rne32(max(abs(v) for v in blk) * k1))
+            inv = rne32(genc / E4M3[e]) if e else Fraction(0)
+            rs.append(e)
+            rc += [e2m1_code(rne32(v * inv), v < 0) for v in blk]
+        codes.append(rc)
+        scales.append(rs)
+    return codes, scales, gdec
+
+
+def pack(codes_row):
+    return [codes_row[2 * j] | (codes_row[2 * j + 1] << 4) for j in range(len(codes_row) // 2)]
+
+
+def test_nvfp4_prepare_chain_is_the_exact_model():
+    """Backbone and residual of a no-norm 2:4 prepare, every fp32 step
+    through the exact model, against the oracle's bytes."""
+    M, K = 2, 256
+    X = wl.activation("laplace_outlier", 98, 0, M, K)
+    R = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4")
+    x = [[bf16(b) for b in row] for row in X]
+    B = []
+    for row in x:
+        out = []
+        for g0 in range(0, K, 4):
+            kp = keep_top2(row[g0:g0 + 4])
+            out += [row[g0 + i] if i in kp else Fraction(0) for i in range(4)]
+        B.append(out)
+    A_b = max(abs(v) for row in x for v in row)
+    bc, bs, bgdec = model_nvfp4(B, A_b)
+    assert [pack(r) for r in bc] == R.bb.codes.tolist()
+    assert bs == R.bb.scales.tolist()
+    assert Fraction(float(R.bb.tscale)) == bgdec
+    # residual r = y - fl(fl(val * s) * G_dec), then its own chain
+    res = []
+    for i, row in enumerate(x):
+        rr = []
+        for k, v in enumerate(row):
+            c = bc[i][k]
+            d = rne32(rne32((-1 if c & 8 else 1) * E2M1[c & 7] * E4M3[bs[i][k // 16]]) * bgdec)
+            rr.append(rne32(v - d))
+        res.append(rr)
+    A_r = max(abs(v) for row in res for v in row)
+    rcodes, rscales, rgdec = model_nvfp4(res, A_r)
+    assert [pack(r) for r in rcodes] == R.rs.codes.tolist()
+    assert rscales == R.rs.scales.tolist()
+    assert Fraction(float(R.rs.tscale)) == rgdec
+
+
+def test_mxfp4_prepare_chain_is_the_exact_model():
+    """MXFP4 backbone: block exponent floor(log2 amax) - 2 (biased 127),
+    element code E2M1(y * 2^-(e-127)), no tensor scale."""
+    M, K = 2, 256
+    X = wl.activation("student_t", 99, 0, M, K)
+    R = oracle.prepare(X, None, 1e-6, 2, 4, "mxfp4")
+    for i, row in enumerate(X):
+        x = [bf16(b) for b in row]
+        out_codes, out_scales = [], []
+        for b0 in range(0, K, 32):
+            blk = x[b0:b0 + 32]
+            kept = []
+            for g0 in range(0, 32, 4):
+                kp = keep_top2(blk[g0:g0 + 4])
+                kept += [blk[g0 + j] if j in kp else Fraction(0) for j in range(4)]
+            amax = max(abs(v) for v in kept)
+            e = 0
+            if amax:
+                fl = amax.numerator.bit_length() - amax.denominator.bit_length()
+                if TWO ** fl > amax:
+                    fl -= 1
+                e = max(fl - 2 + 127, 0)
+            out_scales.append(e)
+            out_codes += [e2m1_code(v * TWO ** (127 - e), v < 0) for v in kept]
+        assert pack(out_codes) == R.bb.codes[i].tolist()
+        assert out_scales == R.bb.scales[i].tolist()
+    assert float(R.bb.tscale) == 1.0
