@@ -162,7 +162,7 @@ WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload(
         "tiny", 1, "normal_outlier",
         (Linear("tiny", 256, 256, True, 0),), Ms=(16,)),
-    # a small SwiGLU MLP (gate+up 256 -> 2 x 128, down 128 -> 256) for the
+    # a small SwiGLU MLP (gate+up 256 -> 2 x 256, down 256 -> 256) for the
     # producer-fused path's quick checks
     "tiny_mlp": Workload(
         "tiny_mlp", 7, "laplace_outlier",
