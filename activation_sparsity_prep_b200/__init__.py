@@ -26,7 +26,7 @@ __all__ = [
     "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
     "prepare", "prepare_layernorm", "prepare_amax", "prepare_noalloc", "linear",
     "linear_swiglu", "interleave_gate_up", "moe_linear", "moe_linear_swiglu",
-    "moe_workspace_bytes", "last_device_status",
+    "moe_workspace_bytes", "selftest_wait_timeout", "last_device_status",
 ]
 
 NVFP4, MXFP4 = 0, 1
@@ -107,6 +107,8 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_moe_linear_swiglu.restype = I
         L.sharq_prepare_noalloc.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P]
         L.sharq_prepare_noalloc.restype = I
+        L.sharq_selftest_wait_timeout.argtypes = [P, I64, P]
+        L.sharq_selftest_wait_timeout.restype = I
         L.sharq_last_device_status.argtypes = [P]
         L.sharq_last_device_status.restype = I
         _lib = L
@@ -393,6 +395,17 @@ def moe_linear_swiglu(x: Prepared, row_index, offsets, w: Weight, out=None, amax
                                      ctypes.byref(cw), H.data_ptr(), a.data_ptr(), ws.data_ptr(),
                                      ws.numel(), _stream(stream)))
     return H, a
+
+
+def selftest_wait_timeout(limit_us: int = 10000, stream=None) -> None:
+    """Run the bounded-wait self-test: a grid wait that one block never
+    joins gives up after limit_us and records a timeout, which the next
+    last_device_status() reports (SHARQ_ERR_TIMEOUT = 4)."""
+    import torch
+    L = load_sharq_ops()
+    ws = torch.zeros((16,), dtype=torch.uint8, device="cuda")
+    _check("sharq_selftest_wait_timeout", L.sharq_selftest_wait_timeout(ws.data_ptr(), int(limit_us),
+                                                                        _stream(stream)))
 
 
 def last_device_status(stream=None) -> int:

@@ -244,6 +244,14 @@ sharq_status sharq_moe_linear_swiglu(const sharq_prepared* x, const int32_t* row
     return moe_common(x, row_index, expert_offsets, E, T, w, H, 0, h_amax, ws, ws_bytes, stream);
 }
 
+sharq_status sharq_selftest_wait_timeout(void* ws, int64_t limit_us, void* stream) {
+    if (!ws || ((uintptr_t)ws & 3u) || limit_us < 1000 || limit_us > 1000000)
+        return SHARQ_ERR_INVALID_ARG;
+    return cuda_status(sharq::launch_wait_selftest(static_cast<uint32_t*>(ws),
+                                                   (unsigned long long)limit_us * 1000ull,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 sharq_status sharq_last_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return SHARQ_ERR_CUDA;

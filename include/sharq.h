@@ -270,6 +270,14 @@ SHARQ_API sharq_status sharq_moe_linear_swiglu(const sharq_prepared* x, const in
 SHARQ_API sharq_status sharq_prepare_noalloc(const void* X_bf16, const void* gamma_bf16, float eps,
                                              const sharq_prepared* out, void* stream);
 
+/* Self-test of the failure path (for test suites): launches a small grid
+ * wait that one block never joins.  Each waiting block gives up after
+ * limit_us microseconds (1000 .. 1000000), records a timeout in the device
+ * status word and returns, so the next sharq_last_device_status() reports
+ * SHARQ_ERR_TIMEOUT and the context stays usable.  ws: device memory of at
+ * least 4 bytes (4-byte aligned), overwritten.  Nothing faults or hangs. */
+SHARQ_API sharq_status sharq_selftest_wait_timeout(void* ws, int64_t limit_us, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word:
  * SHARQ_OK, SHARQ_ERR_TIMEOUT if a bounded device wait gave up since the
  * last call, or SHARQ_ERR_CUDA if the stream itself reports an error. */

@@ -176,3 +176,11 @@ def test_moe_swiglu_needs_an_amax():
 def test_public_api_names_resolve():
     for n in sq.__all__:
         assert hasattr(sq, n), n
+
+
+def test_wait_selftest_rejects_bad_arguments_on_host():
+    L = sq.load_sharq_ops()
+    assert L.sharq_selftest_wait_timeout(None, 10000, None) == 1
+    assert L.sharq_selftest_wait_timeout(0x1002, 10000, None) == 1      # misaligned
+    assert L.sharq_selftest_wait_timeout(0x1000, 10, None) == 1         # below 1 ms
+    assert L.sharq_selftest_wait_timeout(0x1000, 5_000_000, None) == 1  # above 1 s
