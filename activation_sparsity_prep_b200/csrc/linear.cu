@@ -12,14 +12,15 @@
 // as bf16 (or fp32).  The SwiGLU form (the gate+up projection of an MLP,
 // its weight rows interleaved 64 gate / 64 up per 128-row tile) writes
 // H = silu(gate) * up instead, half as many bf16 columns, and the maximum of
-// |H|: the next prepare's backbone amax, so that prepare skips its own
-// pass over H.  When the two tensor scales are equal by construction
-// (MXFP4, or a residual quantised against the backbone's tensor scale) both
-// MMAs accumulate into one accumulator, Y = G_w * G_b * acc, and the two
+// |H|: the next prepare's backbone amax, so that prepare skips its own pass
+// over H.  When the two tensor scales are equal by construction (MXFP4, or
+// a residual quantised against the backbone's tensor scale) both MMAs
+// accumulate into one accumulator, Y = G_w * G_b * acc, and the two
 // tensor-memory accumulators serve as a double buffer instead: the next
-// tile's MMAs run while the epilogue drains the previous one.  The backbone runs as a dense MMA over zero-filled codes:
-// the FP4 sparse MMA carries one scale per 32 logical elements, which cannot
-// express NVFP4's per-16 backbone scales.
+// tile's MMAs run while the epilogue drains the previous one.  The backbone
+// runs as a dense MMA over zero-filled codes: the FP4 sparse MMA carries one
+// scale per 32 logical elements, which cannot express NVFP4's per-16
+// backbone scales.
 //
 // CTA layout (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
 // and MMA issuer, warps 2..5 = epilogue (one TMEM lane quarter each),
