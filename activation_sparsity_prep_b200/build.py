@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsharq.so")
-SOURCES = ["abi.cu", "prepare.cu", "linear.cu", "noalloc.cu"]
+SOURCES = ["abi.cu", "prepare.cu", "linear.cu", "noalloc.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "sharq_internal.h"]
 
 NVCC_FLAGS = [

@@ -255,7 +255,8 @@ sharq_status sharq_selftest_wait_timeout(void* ws, int64_t limit_us, void* strea
 sharq_status sharq_last_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return SHARQ_ERR_CUDA;
-    unsigned v = sharq::take_status_prepare() | sharq::take_status_linear();
+    unsigned v = sharq::take_status_prepare() | sharq::take_status_linear() |
+                 sharq::take_status_selftest();
     if (v & sharq::kStatusReadFailed) return SHARQ_ERR_CUDA;
     if (v & (sharq::kStatusGridTimeout | sharq::kStatusMbarTimeout)) return SHARQ_ERR_TIMEOUT;
     if (v) return SHARQ_ERR_CUDA;

@@ -696,36 +696,6 @@ cudaError_t launch_m(const PrepArgs& a, int m, cudaStream_t s, int sms) {
 
 }  // namespace
 
-namespace {
-
-// Self-test of the bounded grid wait (the wait of grid_barrier, with a
-// caller-chosen limit): every block but the last arrives on *counter and
-// waits for all gridDim.x arrivals.  The last block never arrives, so each
-// wait runs out after limit_ns, records the timeout bit and returns --
-// the path a real barrier takes when a block is lost, without hanging.
-__global__ void __launch_bounds__(32) wait_selftest_kernel(uint32_t* counter,
-                                                            unsigned long long limit_ns) {
-    if (blockIdx.x == gridDim.x - 1 || threadIdx.x != 0) return;
-    atomicAdd(counter, 1u);
-    const unsigned long long t0 = globaltimer();
-    while (ld_acquire_gpu(counter) < gridDim.x) {
-        if (globaltimer() - t0 > limit_ns) {
-            record_status(kStatusGridTimeout);
-            break;
-        }
-        __nanosleep(256);
-    }
-}
-
-}  // namespace
-
-cudaError_t launch_wait_selftest(uint32_t* counter, unsigned long long limit_ns, cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(uint32_t), s);
-    if (e != cudaSuccess) return e;
-    wait_selftest_kernel<<<4, 32, 0, s>>>(counter, limit_ns);
-    return cudaGetLastError();
-}
-
 size_t prepare_ws_bytes(int64_t M) {
     size_t b = 64 + (size_t)(M > 0 ? M : 0) * 8;
     return (b + 255) / 256 * 256;

@@ -33,7 +33,8 @@ struct PrepareLaunch {
 
 size_t prepare_ws_bytes(int64_t M);
 cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms);
-// Failure-path self-test: a grid wait that one block never joins, bounded by limit_ns.
+// Failure-path self-test (selftest.cu): a grid wait that one block never
+// joins, bounded by limit_ns.
 cudaError_t launch_wait_selftest(uint32_t* counter, unsigned long long limit_ns, cudaStream_t s);
 
 struct LinearLaunch {
@@ -73,5 +74,6 @@ int device_sm_count();
 // Read and clear the device status words of each kernel file.
 unsigned take_status_prepare();
 unsigned take_status_linear();
+unsigned take_status_selftest();
 
 }  // namespace sharq
