@@ -333,6 +333,88 @@ def moe_linear(prep: Prepared, row_index: np.ndarray, offsets: np.ndarray,
     return Y
 
 
+# ----------------------------------------- pair-granular 4:8 backbone ----
+# The FP4 sparse tensor-core MMA takes its sparse operand as kept PAIRS of
+# FP4 elements: two of the four aligned pairs of every eight elements, with
+# a 2-bit pair index each.  An input-adaptive mask of that shape (SharQ
+# paper, Abstract: the N:M mask is chosen per input) keeps, in every aligned
+# group of eight, the two pairs of largest magnitude.  Reading: a pair's
+# magnitude is max(|y_2i|, |y_2i+1|), so the pair holding the group's largest
+# entry is always kept (the backbone's block maxima stay those of y); ties go
+# to the lower pair index.  The backbone format is MXFP4, whose per-32
+# scales the sparse MMA can carry (NVFP4's per-16 scales it cannot).
+
+def mask_pairs(y: np.ndarray) -> np.ndarray:
+    """0/1 keep flags [M, K] of the pair-granular 4:8 mask of y [M, K]."""
+    y = np.asarray(y, dtype=np.float32)
+    M, K = y.shape
+    if K % 8:
+        raise ValueError("K must be a multiple of 8")
+    mag = np.abs(y).reshape(M, K // 8, 4, 2).max(axis=3)          # [M, G, 4] pair magnitudes
+    keep_pair = np.zeros((M, K // 8, 4), dtype=np.uint8)
+    for i in range(4):
+        beaten_by = np.zeros((M, K // 8), dtype=np.int32)
+        for j in range(4):
+            if j == i:
+                continue
+            # j outranks i: larger magnitude, or equal and a lower index
+            beaten_by += (mag[:, :, j] > mag[:, :, i]) | ((mag[:, :, j] == mag[:, :, i]) & (j < i))
+        keep_pair[:, :, i] = beaten_by < 2
+    return np.repeat(keep_pair, 2, axis=2).reshape(M, K)
+
+
+def compress_pairs(codes: np.ndarray, keep: np.ndarray):
+    """Zero-filled packed E2M1 codes [M, K/2] and their pair mask -> (kept
+    codes [M, K/4]: the two kept pairs of every group of eight in order, one
+    byte per pair; pair indices [M, K/8]: the two 2-bit indices of every group,
+    lower kept pair in bits 1:0, higher in bits 3:2)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    M, K2 = codes.shape
+    K = 2 * K2
+    kp = np.asarray(keep, dtype=np.int32).reshape(M, K // 8, 4, 2)[:, :, :, 0]   # [M, G, 4]
+    if not np.all(kp.sum(axis=2) == 2):
+        raise ValueError("every group of eight must keep exactly two pairs")
+    pairs = codes.reshape(M, K // 8, 4)                            # one byte = one pair
+    idx = np.argsort(-kp, axis=2, kind="stable")[:, :, :2]         # kept pair indices, ascending
+    idx = np.sort(idx, axis=2)
+    kept = np.take_along_axis(pairs, idx, axis=2).reshape(M, K // 4)
+    meta = (idx[:, :, 0] | (idx[:, :, 1] << 2)).astype(np.uint8)
+    return kept.astype(np.uint8), meta
+
+
+def decompress_pairs(kept: np.ndarray, meta: np.ndarray) -> np.ndarray:
+    """Inverse of compress_pairs: the zero-filled packed codes [M, K/2]."""
+    kept = np.asarray(kept, dtype=np.uint8)
+    meta = np.asarray(meta, dtype=np.uint8)
+    M, G = meta.shape
+    out = np.zeros((M, G, 4), dtype=np.uint8)
+    k2 = kept.reshape(M, G, 2)
+    for slot in range(2):
+        idx = (meta >> (2 * slot)) & 3
+        np.put_along_axis(out, idx[:, :, None].astype(np.int64), k2[:, :, slot:slot + 1], axis=2)
+    return out.reshape(M, G * 4)
+
+
+def prepare_pairs(X: np.ndarray, gamma: Optional[np.ndarray], eps: float = 1e-6):
+    """The preparation operator with the pair-granular 4:8 mask and an MXFP4
+    backbone: y = RMSNorm(X) * gamma (or X), keep = mask_pairs(y), the
+    backbone B = keep ? y : 0 quantised to MXFP4 (its zero-filled codes and
+    their compressed form), and the residual y - dequant(B) quantised to
+    MXFP4.  Returns (Prepared with the zero-filled backbone, kept codes,
+    pair indices)."""
+    y = normalize(X, gamma, eps)
+    keep = mask_pairs(y)
+    B = np.where(keep == 1, y, np.float32(0.0)).astype(np.float32)
+    bq = quantize(B, "mxfp4", want_D=True)
+    r = (y - bq.D).astype(np.float32)                               # one fp32 subtraction each
+    rq = quantize(r, "mxfp4")
+    M, K = y.shape
+    mbits = np.packbits(keep.reshape(M, K // 8, 8), axis=2, bitorder="little").reshape(M, K // 8)
+    kept, meta = compress_pairs(bq.codes, keep)
+    bq.D = None
+    return Prepared(mbits, bq, rq, 4, 8, MXFP4, y, r), kept, meta
+
+
 # ------------------------------------------------ producer-fused MLP ----
 # SharQ paper, Abstract: the preparation is one operator in front of each
 # FP4 linear.  For a SwiGLU MLP the down projection's input is
