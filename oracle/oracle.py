@@ -366,8 +366,10 @@ def mask_pairs(y: np.ndarray) -> np.ndarray:
 def compress_pairs(codes: np.ndarray, keep: np.ndarray):
     """Zero-filled packed E2M1 codes [M, K/2] and their pair mask -> (kept
     codes [M, K/4]: the two kept pairs of every group of eight in order, one
-    byte per pair; pair indices [M, K/8]: the two 2-bit indices of every group,
-    lower kept pair in bits 1:0, higher in bits 3:2)."""
+    byte per pair; pair indices [M, K/16]: per group of eight a nibble with
+    the lower kept pair's 2-bit index in bits 1:0 and the higher one's in
+    bits 3:2, group 2j in the low nibble of byte j -- the row-major
+    metadata the FP4 sparse MMA reads, 4 bits per 8 logical elements)."""
     codes = np.asarray(codes, dtype=np.uint8)
     M, K2 = codes.shape
     K = 2 * K2
@@ -378,7 +380,8 @@ def compress_pairs(codes: np.ndarray, keep: np.ndarray):
     idx = np.argsort(-kp, axis=2, kind="stable")[:, :, :2]         # kept pair indices, ascending
     idx = np.sort(idx, axis=2)
     kept = np.take_along_axis(pairs, idx, axis=2).reshape(M, K // 4)
-    meta = (idx[:, :, 0] | (idx[:, :, 1] << 2)).astype(np.uint8)
+    nib = (idx[:, :, 0] | (idx[:, :, 1] << 2)).astype(np.uint8)          # [M, K/8]
+    meta = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)          # [M, K/16]
     return kept.astype(np.uint8), meta
 
 
@@ -386,11 +389,13 @@ def decompress_pairs(kept: np.ndarray, meta: np.ndarray) -> np.ndarray:
     """Inverse of compress_pairs: the zero-filled packed codes [M, K/2]."""
     kept = np.asarray(kept, dtype=np.uint8)
     meta = np.asarray(meta, dtype=np.uint8)
-    M, G = meta.shape
+    M = meta.shape[0]
+    nib = np.stack([meta & 0xF, meta >> 4], axis=2).reshape(M, -1)        # [M, K/8]
+    G = nib.shape[1]
     out = np.zeros((M, G, 4), dtype=np.uint8)
     k2 = kept.reshape(M, G, 2)
     for slot in range(2):
-        idx = (meta >> (2 * slot)) & 3
+        idx = (nib >> (2 * slot)) & 3
         np.put_along_axis(out, idx[:, :, None].astype(np.int64), k2[:, :, slot:slot + 1], axis=2)
     return out.reshape(M, G * 4)
 

@@ -62,15 +62,17 @@ def test_mask_pairs_invariants():
 def test_compress_round_trip_and_layout():
     X = wl.activation("student_t", 72, 0, 5, 256)
     P, kept, meta = oracle.prepare_pairs(X, None)
-    assert kept.shape == (5, 64) and meta.shape == (5, 32)
+    assert kept.shape == (5, 64) and meta.shape == (5, 16)
     assert np.array_equal(oracle.decompress_pairs(kept, meta), P.bb.codes)
-    lo, hi = meta & 3, meta >> 2
-    assert np.all(lo < hi) and np.all(hi < 4)
-    # hand-made group: pairs 1 and 3 kept
-    codes = np.array([[0x00, 0x21, 0x00, 0x9F]], dtype=np.uint8)
-    keep = np.array([[0, 0, 1, 1, 0, 0, 1, 1]], dtype=np.uint8)
+    for nib in (meta & 0xF, meta >> 4):
+        lo, hi = nib & 3, nib >> 2
+        assert np.all(lo < hi) and np.all(hi < 4)
+    # hand-made groups: pairs 1 and 3 kept, then pairs 0 and 2
+    codes = np.array([[0x00, 0x21, 0x00, 0x9F, 0x7A, 0x00, 0x05, 0x00]], dtype=np.uint8)
+    keep = np.array([[0, 0, 1, 1, 0, 0, 1, 1, 1, 1, 0, 0, 1, 1, 0, 0]], dtype=np.uint8)
     k, m = oracle.compress_pairs(codes, keep)
-    assert k.tolist() == [[0x21, 0x9F]] and m.tolist() == [[1 | (3 << 2)]]
+    assert k.tolist() == [[0x21, 0x9F, 0x7A, 0x05]]
+    assert m.tolist() == [[(1 | (3 << 2)) | ((0 | (2 << 2)) << 4)]]
 
 
 def test_prepare_pairs_reconstructs_and_shares_block_scales():
