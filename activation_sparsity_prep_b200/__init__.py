@@ -141,6 +141,87 @@ def _check(fn: str, st: int):
         raise SharqError(fn, st)
 
 
+
+# ------------------------------------------------------- argument checks --
+# The C ABI sees raw pointers only, so a tensor of the wrong shape, dtype or
+# device would be read or written past its end on the GPU.  Every wrapper
+# checks its tensors here first and raises ValueError.
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_tensor(name: str, t, shape, dtype, device=None):
+    """t must be a contiguous tensor of exactly `shape` and `dtype` on
+    `device` (when given)."""
+    _need(t is not None, f"{name} is required")
+    _need(tuple(t.shape) == tuple(shape), f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    _need(t.dtype == dtype, f"{name} has dtype {t.dtype}, expected {dtype}")
+    _need(t.is_contiguous(), f"{name} must be contiguous")
+    if device is not None:
+        _need(t.device == device, f"{name} is on {t.device}, expected {device}")
+
+
+def _check_min(name: str, t, numel: int, dtype, device):
+    """A flat buffer of at least `numel` elements of `dtype` on `device`."""
+    _need(t is not None, f"{name} is required")
+    _need(t.dtype == dtype, f"{name} has dtype {t.dtype}, expected {dtype}")
+    _need(t.is_contiguous(), f"{name} must be contiguous")
+    _need(t.numel() >= numel, f"{name} holds {t.numel()} elements, needs {numel}")
+    _need(t.device == device, f"{name} is on {t.device}, expected {device}")
+
+
+def _check_input(X, gamma=None, beta=None):
+    """X bf16 [M, K] on a CUDA device; gamma / beta bf16 [K] beside it."""
+    import torch
+    _need(X is not None and X.dim() == 2, "X must be a 2-D tensor [M, K]")
+    _need(X.is_cuda, "X must be a CUDA tensor")
+    _check_tensor("X", X, X.shape, torch.bfloat16)
+    K = X.shape[1]
+    for nm, v in (("gamma", gamma), ("beta", beta)):
+        if v is not None:
+            _check_tensor(nm, v, (K,), torch.bfloat16, X.device)
+
+
+def _check_prepared(p: "Prepared", M: int, K: int, fmt: int, device):
+    """A caller-given Prepared must describe [M, K] in `fmt` with buffers
+    large enough for it, on `device`."""
+    import torch
+    _need((p.M, p.K, p.fmt) == (M, K, fmt),
+          f"out describes M={p.M}, K={p.K}, fmt={p.fmt}; the call needs M={M}, K={K}, fmt={fmt}")
+    _check_prepared_buffers(p, device)
+
+
+def _check_prepared_buffers(p: "Prepared", device=None):
+    import torch
+    dev = device if device is not None else p.bb_codes.device
+    sb = scale_bytes(p.M, p.K, p.fmt)
+    u8 = torch.uint8
+    _check_min("bb_codes", p.bb_codes, p.M * p.K // 2, u8, dev)
+    _check_min("rs_codes", p.rs_codes, p.M * p.K // 2, u8, dev)
+    _check_min("bb_scales", p.bb_scales, sb, u8, dev)
+    _check_min("rs_scales", p.rs_scales, sb, u8, dev)
+    _check_min("bb_tscale", p.bb_tscale, 1, torch.float32, dev)
+    _check_min("rs_tscale", p.rs_tscale, 1, torch.float32, dev)
+    if p.mask is not None:
+        _check_min("mask", p.mask, p.M * p.K // 8, u8, dev)
+    return dev
+
+
+def _check_weight(w: "Weight", K: int, fmt: int, device, E: int = 1):
+    import torch
+    _need(w.K == K, f"weight K={w.K} does not match the activations' K={K}")
+    _need(w.fmt == fmt, f"weight format {w.fmt} does not match the activations' {fmt}")
+    _check_min("weight codes", w.codes, E * w.N * K // 2, torch.uint8, device)
+    _check_min("weight scales", w.scales, E * scale_bytes(w.N, K, fmt), torch.uint8, device)
+    _check_min("weight tensor_scale", w.tensor_scale, E, torch.float32, device)
+
+
+def _check_output(name: str, Y, shape, dtype, device):
+    _check_tensor(name, Y, shape, dtype, device)
+
+
 def scale_bytes(rows: int, K: int, fmt="nvfp4") -> int:
     return int(load_sharq_ops().sharq_scale_bytes(rows, K, _fmt(fmt)))
 
@@ -224,8 +305,12 @@ def _workspace(M: int, K: int, fmt: int, ws=None, device="cuda"):
 def quantize_weight(W, fmt="nvfp4", out: Optional[Weight] = None, ws=None, stream=None) -> Weight:
     """W: bf16 [N, K] device tensor -> shared FP4 payload."""
     L = load_sharq_ops()
+    _check_input(W)
     N, K = W.shape
     f = _fmt(fmt)
+    if out is not None:
+        _need((out.N, out.K, out.fmt) == (N, K, f), "out does not describe W's shape and format")
+        _check_weight(out, K, f, W.device)
     w = out if out is not None else Weight.empty(N, K, f, device=W.device)
     ws = _workspace(N, K, f, ws, W.device)
     cw = w._c()
@@ -242,8 +327,11 @@ def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4
     residual_scale: "own" or "shared" (ignored when ``out`` is given: the
     output's own setting applies)."""
     L = load_sharq_ops()
+    _check_input(X, gamma)
     M, K = X.shape
     f = _fmt(fmt)
+    if out is not None:
+        _check_prepared(out, M, K, f, X.device)
     p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
                                                    residual_scale=residual_scale)
     ws = _workspace(M, K, f, ws, X.device)
@@ -260,8 +348,11 @@ def prepare_layernorm(X, gamma, beta=None, eps: float = 1e-6, n: int = 2, m: int
     """prepare() with LayerNorm (gamma required, beta optional) instead of
     RMSNorm in front of the mask."""
     L = load_sharq_ops()
+    _check_input(X, gamma, beta)
     M, K = X.shape
     f = _fmt(fmt)
+    if out is not None:
+        _check_prepared(out, M, K, f, X.device)
     p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
                                                    residual_scale=residual_scale)
     ws = _workspace(M, K, f, ws, X.device)
@@ -281,8 +372,11 @@ def prepare_noalloc(X, gamma=None, eps: float = 1e-6, out: Optional[Prepared] = 
     (fixed in-library scratch, M <= NOALLOC_MAX_ROWS).  The output buffers
     are the caller's: pass ``out`` when the caller cannot allocate either."""
     L = load_sharq_ops()
+    _check_input(X, gamma)
     M, K = X.shape
     f = _fmt(fmt)
+    if out is not None:
+        _check_prepared(out, M, K, f, X.device)
     p = out if out is not None else Prepared.empty(M, K, n, m, f, device=X.device)
     cp = p._c()
     _check("sharq_prepare_noalloc",
@@ -295,8 +389,12 @@ def linear(x: Prepared, w: Weight, out_fp32: bool = False, out=None, stream=None
     """Two-path FP4 linear: Y = G_w (G_b A_b W^T + G_r A_r W^T)."""
     import torch
     L = load_sharq_ops()
+    dev = _check_prepared_buffers(x)
+    _check_weight(w, x.K, x.fmt, dev)
     dt = torch.float32 if out_fp32 else torch.bfloat16
-    Y = out if out is not None else torch.empty((x.M, w.N), dtype=dt, device=x.bb_codes.device)
+    if out is not None:
+        _check_output("out", out, (x.M, w.N), dt, dev)
+    Y = out if out is not None else torch.empty((x.M, w.N), dtype=dt, device=dev)
     cx, cw = x._c(), w._c()
     _check("sharq_linear", L.sharq_linear(ctypes.byref(cx), ctypes.byref(cw), Y.data_ptr(),
                                           1 if out_fp32 else 0, _stream(stream)))
@@ -319,7 +417,12 @@ def linear_swiglu(x: Prepared, w: Weight, out=None, amax=None, stream=None):
     amax fp32 [1] = max |H|), for w quantised from interleave_gate_up(...)."""
     import torch
     L = load_sharq_ops()
-    dev = x.bb_codes.device
+    dev = _check_prepared_buffers(x)
+    _check_weight(w, x.K, x.fmt, dev)
+    if out is not None:
+        _check_output("out", out, (x.M, w.N // 2), torch.bfloat16, dev)
+    if amax is not None:
+        _check_output("amax", amax, (1,), torch.float32, dev)
     H = out if out is not None else torch.empty((x.M, w.N // 2), dtype=torch.bfloat16, device=dev)
     a = amax if amax is not None else torch.empty((1,), dtype=torch.float32, device=dev)
     cx, cw = x._c(), w._c()
@@ -333,16 +436,39 @@ def prepare_amax(X, amax, n: int = 2, m: int = 4, fmt="nvfp4", want_mask: bool =
     """prepare() of a no-norm input whose max |X| the producer has already
     taken (amax: fp32 [1] device tensor, e.g. from linear_swiglu)."""
     L = load_sharq_ops()
+    _check_input(X)
     M, K = X.shape
     f = _fmt(fmt)
+    if out is not None:
+        _check_prepared(out, M, K, f, X.device)
     p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
                                                    residual_scale=residual_scale)
+    import torch
+    _check_tensor("amax", amax, (1,), torch.float32, X.device)
     ws = _workspace(M, K, f, ws, X.device)
     cp = p._c()
     _check("sharq_prepare_amax",
            L.sharq_prepare_amax(X.data_ptr(), amax.data_ptr(), ctypes.byref(cp), ws.data_ptr(),
                                 ws.numel(), _stream(stream)))
     return p
+
+
+def _check_grouped(x: Prepared, row_index, offsets, w: Weight, T: int):
+    """Shapes of the grouped form's index arrays and stacked weight; returns
+    the device."""
+    import torch
+    dev = _check_prepared_buffers(x)
+    _need(offsets is not None and offsets.dim() == 1 and offsets.numel() >= 2,
+          "offsets must be an int32 [E+1] tensor with E >= 1")
+    E = int(offsets.numel()) - 1
+    _check_tensor("offsets", offsets, (E + 1,), torch.int32, dev)
+    if row_index is not None:
+        _check_tensor("row_index", row_index, (T,), torch.int32, dev)
+    else:
+        _need(T == x.M, f"without row_index the dispatched rows are the prepared rows: T={T}, M={x.M}")
+    _need(w.E == E, f"the weight stacks {w.E} experts, offsets describe {E}")
+    _check_weight(w, x.K, x.fmt, dev, E)
+    return dev
 
 
 def moe_workspace_bytes(T: int, E: int, K: int, fmt="nvfp4") -> int:
@@ -360,7 +486,9 @@ def moe_linear(x: Prepared, row_index, offsets, w: Weight, out_fp32: bool = Fals
         T = int(row_index.numel()) if row_index is not None else x.M
     E = int(offsets.numel()) - 1
     dt = torch.float32 if out_fp32 else torch.bfloat16
-    dev = x.bb_scales.device
+    dev = _check_grouped(x, row_index, offsets, w, T)
+    if out is not None:
+        _check_output("out", out, (T, w.N), dt, dev)
     Y = out if out is not None else torch.empty((T, w.N), dtype=dt, device=dev)
     need = moe_workspace_bytes(T, E, x.K, x.fmt)
     if ws is None or ws.numel() < need:
@@ -383,7 +511,11 @@ def moe_linear_swiglu(x: Prepared, row_index, offsets, w: Weight, out=None, amax
     if T is None:
         T = int(row_index.numel()) if row_index is not None else x.M
     E = int(offsets.numel()) - 1
-    dev = x.bb_scales.device
+    dev = _check_grouped(x, row_index, offsets, w, T)
+    if out is not None:
+        _check_output("out", out, (T, w.N // 2), torch.bfloat16, dev)
+    if amax is not None:
+        _check_output("amax", amax, (1,), torch.float32, dev)
     H = out if out is not None else torch.empty((T, w.N // 2), dtype=torch.bfloat16, device=dev)
     a = amax if amax is not None else torch.empty((1,), dtype=torch.float32, device=dev)
     need = moe_workspace_bytes(T, E, x.K, x.fmt)

@@ -1,12 +1,16 @@
 #!/usr/bin/env python
 """Benchmark of the SharQ hot path on B200.
 
-One step = the four linears of a Llama-3.1-8B-shaped decoder layer (qkv,
-o, gate+up, down) at prefill M = 2048 tokens, each run as the fused
-prepare (RMSNorm + 2:4 mask + NVFP4 backbone + NVFP4 residual) followed by
-the two-path tcgen05 FP4 linear.  Weights are quantised once, outside the
-timed region.  Inputs are seeded synthetic tensors (Laplace activations with
-0.5 % outlier channels, N(0, 0.02) weights).
+One step (default) = the three linears of a Qwen2.5-7B-shaped decoder
+layer (qkv 3584 -> 4608, gate+up 3584 -> 37888, down 18944 -> 3584) at
+prefill M = 4096 tokens, each run as the fused prepare (RMSNorm on qkv and
+gate+up + 2:4 mask + NVFP4 backbone + NVFP4 residual with its own tensor
+scale) followed by the two-path tcgen05 FP4 linear.  Weights are quantised
+once, outside the timed region.  Inputs are seeded synthetic tensors
+(Student-t(3) activations with a LogNormal(0, 0.5) per-token scale,
+N(0, 0.02) weights).  ``--workload`` selects the other shapes (Llama-3.1-8B
+linears at M in {1, 16, 128, 2048}, the Qwen3-30B-A3B expert layer, the
+format/mask sweep at M = 16384, a LayerNorm DiT block).
 
 Metric: effective TFLOP/s = sum over linears of 2*M*N*K / step time; the
 JSON line also carries tokens/s, the roofline of the dominant kernel (the
@@ -52,7 +56,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
-    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--workload", default="qwen7b")
     ap.add_argument("--M", type=int, default=None,
                     help="rows per linear (default: 2048 for llama8b, the workload's own M otherwise)")
     ap.add_argument("--fmt", default="nvfp4")
@@ -307,6 +311,14 @@ def moe_reference_sample(W, fmt, tokens: int = 4, fuse_mlp=False):
     return sample
 
 
+def host_cores():
+    """CPU cores this process may run on (its affinity set)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def blas_threads():
     try:
         import threadpoolctl
@@ -316,24 +328,42 @@ def blas_threads():
         return 1
 
 
-def cpu_baseline(linears, args, budget_s: float = 15.0, rows: int = 16):
+def cpu_baseline(linears, args, budget_s: float = 10.0, rows: int = 16):
+    """The oracle timed on the host over a bounded sample (the first `rows`
+    rows of every linear): once with the BLAS pool at its default size and
+    once with one thread, about `budget_s` seconds each."""
     import oracle
     n_, m_ = nm_of(args)
     quantized = [oracle.quantize_weight(gate_up_interleaved(d["W"]) if args.fuse_mlp and L.name == "gate_up"
                                         else d["W"], args.fmt) for L, d in linears]
-    total_t, total_f, n = 0.0, 0.0, 0
-    while total_t < budget_s and n < 50:
-        t, f = oracle_sample_step(linears, rows, quantized, args.fmt, n_, m_, args.residual,
-                                  args.fuse_mlp)
-        total_t += t
-        total_f += f
-        n += 1
-    return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-            "kind": "oracle",
+
+    def timed():
+        total_t, total_f, n = 0.0, 0.0, 0
+        while total_t < budget_s and n < 50:
+            t, f = oracle_sample_step(linears, rows, quantized, args.fmt, n_, m_, args.residual,
+                                      args.fuse_mlp)
+            total_t += t
+            total_f += f
+            n += 1
+        return total_f / total_t / 1e12, n
+
+    threads = blas_threads()
+    value, n = timed()
+    one = None
+    try:
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(limits=1, user_api="blas"):
+            one, _ = timed()
+    except Exception:
+        pass
+    return {"value": value, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+            "threads": {"gemm_blas": threads, "prepare": 1},
+            "single_thread_value": one,
             "sample": f"{n} passes of: oracle prepare + fp64 two-path linear on the first {rows} "
                       f"rows of each of the {len(linears)} linears (all N"
                       f"{'; SwiGLU of gate+up feeds down' if args.fuse_mlp else ''}); prepare "
-                      f"single-threaded C, GEMM numpy/OpenBLAS fp64"}
+                      f"single-threaded C, GEMM numpy/OpenBLAS fp64 on {threads} threads "
+                      f"(single_thread_value: the same sample with one BLAS thread)"}
 
 
 def workload_desc(W, M):
@@ -363,7 +393,8 @@ def run_reference(args):
         return 0
     W = wl.WORKLOADS[args.workload]
     n, m = nm_of(args)
-    cores = blas_threads()
+    cores = host_cores()
+    threads = blas_threads()
     if W.moe is None:
         linears = make_inputs(W, args.M)
         import oracle
@@ -399,7 +430,9 @@ def run_reference(args):
         "data": "synthetic",
         "config": bench_config(args, W, M),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": what + "; prepare single-threaded C, GEMM numpy/OpenBLAS fp64"},
+                         "threads": {"gemm_blas": threads, "prepare": 1},
+                         "sample": what + f"; prepare single-threaded C, GEMM numpy/OpenBLAS fp64 "
+                                          f"on {threads} threads"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

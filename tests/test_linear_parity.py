@@ -10,8 +10,10 @@ Tolerances:
   paths share one (MXFP4, or a residual with the backbone's tensor scale).
 * bf16 output: within one bf16 ulp of RNE(Y64); where cancellation makes
   gamma * A larger than half an ulp (no fp32 accumulation can do better
-  there), within one ulp plus gamma * A.  The number of such elements is
-  reported."""
+  there), within one ulp plus gamma * A.  Such elements must stay rare: at
+  most WIDE_CAP of the elements compared (cancellation to below half an
+  ulp of the magnitude sum happens at a few elements per million on these
+  inputs)."""
 import numpy as np
 import pytest
 import torch
@@ -24,6 +26,7 @@ from tests.sharq_testlib import canonical_to_atoms, to_dev, to_np
 pytestmark = pytest.mark.gpu
 
 FROB_TOL = 1e-5
+WIDE_CAP = 1e-3      # fraction of elements allowed to need the cancellation widening
 
 
 def bf16_ordered(b):
@@ -81,6 +84,8 @@ def check(Y32, Ybf, Y64, A, K, rows=None, one_acc=False):
         f"{int((~strict).sum())} elements beyond 1 bf16 ulp, {int((~(strict | widened)).sum())} beyond the widened bound"
     n_wide = int((~strict).sum())
     print(f"rel. Frobenius {err:.2e}; {n_wide} of {d.size} elements need the cancellation widening")
+    assert n_wide <= WIDE_CAP * d.size, \
+        f"{n_wide} of {d.size} elements need the cancellation widening (cap {WIDE_CAP:g})"
     return err, n_wide
 
 

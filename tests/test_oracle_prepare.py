@@ -365,3 +365,57 @@ def test_shared_residual_tensor_scale_is_the_backbones():
     a = oracle.prepare(X, None, 1e-6, 2, 4, "mxfp4", residual_scale="own")
     b = oracle.prepare(X, None, 1e-6, 2, 4, "mxfp4", residual_scale="shared")
     assert np.array_equal(a.rs.codes, b.rs.codes) and np.array_equal(a.rs.scales, b.rs.scales)
+
+
+def _val_e2m1_bruteforce(codes, i, k):
+    """Decoded E2M1 element k of row i, from the nibble layout and the format
+    table written out here (not the oracle's decoder)."""
+    byte = int(codes[i, k // 2])
+    c = byte & 15 if k % 2 == 0 else byte >> 4
+    return [0, .5, 1, 1.5, 2, 3, 4, 6][c & 7] * (-1.0 if c & 8 else 1.0)
+
+
+def _scale_bruteforce(scales, fmt, i, k):
+    """Block scale of element k of row i: E4M3 per 16 (bias 7, subnormals
+    m * 2^-9) or E8M0 per 32 (2^(c - 127)), from the bit fields."""
+    if fmt == "nvfp4":
+        c = int(scales[i, k // 16])
+        e, m = (c >> 3) & 15, c & 7
+        return m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+    return 2.0 ** (int(scales[i, k // 32]) - 127)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("residual", ["own", "shared"])
+def test_linear_abs_bruteforce_tiny(fmt, residual):
+    """linear_abs sets the width of the GPU parity tolerance, so it is pinned
+    from both sides: it must EQUAL the magnitude sum
+    G_w (G_b sum_k |b_ik w_jk| + G_r sum_k |r_ik w_jk|), evaluated here index
+    by index with its own decoder.  A tensor scale applied twice, a missing
+    absolute value or a swapped operand would all change it."""
+    X = wl.activation("laplace_outlier", 2, 7, 3, 128)
+    W = wl.weight(2, 7, 5, 128)
+    P = oracle.prepare(X, wl.gamma_ones(128), 1e-6, 2, 4, fmt, residual_scale=residual)
+    Wq = oracle.quantize_weight(W, fmt)
+    A = oracle.linear_abs(P, Wq)
+    Y = oracle.linear(P, Wq)
+    assert A.shape == (3, 5)
+    for i in range(3):
+        for j in range(5):
+            ab = ar = yb = yr = 0.0
+            for k in range(128):
+                w = _val_e2m1_bruteforce(Wq.codes, j, k) * _scale_bruteforce(Wq.scales, fmt, j, k)
+                b = _val_e2m1_bruteforce(P.bb.codes, i, k) * _scale_bruteforce(P.bb.scales, fmt, i, k)
+                r = _val_e2m1_bruteforce(P.rs.codes, i, k) * _scale_bruteforce(P.rs.scales, fmt, i, k)
+                ab += abs(b * w)
+                ar += abs(r * w)
+                yb += b * w
+                yr += r * w
+            gw, gb, gr = float(Wq.tscale), float(P.bb.tscale), float(P.rs.tscale)
+            want = gw * (gb * ab + gr * ar)
+            assert abs(A[i, j] - want) <= 1e-12 * want
+            # the bound holds the signed result and is not slack by a constant
+            assert abs(Y[i, j]) <= A[i, j] * (1 + 1e-12)
+            assert abs(Y[i, j] - gw * (gb * yb + gr * yr)) <= 1e-12 * want
+    # both paths contribute (neither half of the sum was dropped)
+    assert np.abs(P.rs.codes & 0x77).sum() > 0 and np.abs(P.bb.codes & 0x77).sum() > 0
