@@ -11,9 +11,9 @@ Tolerances:
 * bf16 output: within one bf16 ulp of RNE(Y64); where cancellation makes
   gamma * A larger than half an ulp (no fp32 accumulation can do better
   there), within one ulp plus gamma * A.  Such elements must stay rare: at
-  most WIDE_CAP of the elements compared (cancellation to below half an
-  ulp of the magnitude sum happens at a few elements per million on these
-  inputs)."""
+  most WIDE_CAP of the elements compared, and never more than WIDE_FLOOR
+  in a small case (measured on B200: at most 2 elements per case, a
+  fraction of at most 3.0e-5, over every linear and grouped case here)."""
 import numpy as np
 import pytest
 import torch
@@ -26,7 +26,8 @@ from tests.sharq_testlib import canonical_to_atoms, to_dev, to_np
 pytestmark = pytest.mark.gpu
 
 FROB_TOL = 1e-5
-WIDE_CAP = 1e-3      # fraction of elements allowed to need the cancellation widening
+WIDE_CAP = 1e-4      # fraction of elements allowed to need the cancellation widening
+WIDE_FLOOR = 4       # ... or this many, whichever is larger
 
 
 def bf16_ordered(b):
@@ -84,8 +85,8 @@ def check(Y32, Ybf, Y64, A, K, rows=None, one_acc=False):
         f"{int((~strict).sum())} elements beyond 1 bf16 ulp, {int((~(strict | widened)).sum())} beyond the widened bound"
     n_wide = int((~strict).sum())
     print(f"rel. Frobenius {err:.2e}; {n_wide} of {d.size} elements need the cancellation widening")
-    assert n_wide <= WIDE_CAP * d.size, \
-        f"{n_wide} of {d.size} elements need the cancellation widening (cap {WIDE_CAP:g})"
+    assert n_wide <= max(WIDE_FLOOR, WIDE_CAP * d.size), \
+        f"{n_wide} of {d.size} elements need the cancellation widening (cap {WIDE_CAP:g}, floor {WIDE_FLOOR})"
     return err, n_wide
 
 
