@@ -26,7 +26,7 @@ __all__ = [
     "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
     "prepare", "prepare_layernorm", "prepare_amax", "prepare_noalloc", "linear",
     "linear_swiglu", "interleave_gate_up", "moe_linear", "moe_linear_swiglu",
-    "moe_workspace_bytes", "selftest_wait_timeout", "last_device_status",
+    "moe_workspace_bytes", "selftest_wait_timeout", "selftest_prepare_timeout", "last_device_status",
 ]
 
 NVFP4, MXFP4 = 0, 1
@@ -109,6 +109,8 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_prepare_noalloc.restype = I
         L.sharq_selftest_wait_timeout.argtypes = [P, I64, P]
         L.sharq_selftest_wait_timeout.restype = I
+        L.sharq_selftest_prepare_timeout.argtypes = [P, ctypes.POINTER(_Prepared), P, SZ, I64, P]
+        L.sharq_selftest_prepare_timeout.restype = I
         L.sharq_last_device_status.argtypes = [P]
         L.sharq_last_device_status.restype = I
         _lib = L
@@ -538,6 +540,23 @@ def selftest_wait_timeout(limit_us: int = 10000, stream=None) -> None:
     ws = torch.zeros((16,), dtype=torch.uint8, device="cuda")
     _check("sharq_selftest_wait_timeout", L.sharq_selftest_wait_timeout(ws.data_ptr(), int(limit_us),
                                                                         _stream(stream)))
+
+
+def selftest_prepare_timeout(X, limit_us: int = 10000, stream=None) -> Prepared:
+    """Run the real NVFP4 prepare of X (no norm, own residual scale) with one
+    block that never arrives at its grid barriers and each barrier wait
+    limited to limit_us: the waits give up and record a timeout, which the
+    next last_device_status() reports.  The returned outputs are unspecified."""
+    L = load_sharq_ops()
+    _check_input(X)
+    M, K = X.shape
+    p = Prepared.empty(M, K, device=X.device)
+    ws = _workspace(M, K, NVFP4, None, X.device)
+    cp = p._c()
+    _check("sharq_selftest_prepare_timeout",
+           L.sharq_selftest_prepare_timeout(X.data_ptr(), ctypes.byref(cp), ws.data_ptr(), ws.numel(),
+                                            int(limit_us), _stream(stream)))
+    return p
 
 
 def last_device_status(stream=None) -> int:

@@ -88,7 +88,8 @@ sharq_status sharq_quantize_weight(const void* W_bf16, const sharq_weight* out, 
 
 static sharq_status prepare_common(const void* X_bf16, const void* gamma_bf16, const void* beta_bf16,
                                    bool layernorm, float eps, const sharq_prepared* out, void* ws,
-                                   size_t ws_bytes, void* stream, const float* amax = nullptr) {
+                                   size_t ws_bytes, void* stream, const float* amax = nullptr,
+                                   unsigned long long wait_ns = 0, int skip_block = -1) {
     if (!out || !ws) return SHARQ_ERR_INVALID_ARG;
     if (layernorm && out->M > 0 && !gamma_bf16) return SHARQ_ERR_INVALID_ARG;
     if (!aligned16(beta_bf16)) return SHARQ_ERR_INVALID_ARG;
@@ -114,6 +115,7 @@ static sharq_status prepare_common(const void* X_bf16, const void* gamma_bf16, c
     p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
     p.rs_codes = o.rs_codes; p.rs_scales = o.rs_scales; p.rs_tscale = o.rs_tscale;
     p.mask = o.mask; p.ws = ws; p.amax = amax;
+    p.wait_ns = wait_ns; p.skip_block = skip_block;
     return cuda_status(sharq::launch_prepare(p, static_cast<cudaStream_t>(stream),
                                              sharq::device_sm_count()));
 }
@@ -250,6 +252,15 @@ sharq_status sharq_selftest_wait_timeout(void* ws, int64_t limit_us, void* strea
     return cuda_status(sharq::launch_wait_selftest(static_cast<uint32_t*>(ws),
                                                    (unsigned long long)limit_us * 1000ull,
                                                    static_cast<cudaStream_t>(stream)));
+}
+
+sharq_status sharq_selftest_prepare_timeout(const void* X_bf16, const sharq_prepared* out, void* ws,
+                                            size_t ws_bytes, int64_t limit_us, void* stream) {
+    if (!out || out->fmt != SHARQ_NVFP4 || out->residual_scale != SHARQ_RESIDUAL_OWN || out->M < 1 ||
+        limit_us < 1000 || limit_us > 1000000)
+        return SHARQ_ERR_INVALID_ARG;
+    return prepare_common(X_bf16, nullptr, nullptr, false, 0.0f, out, ws, ws_bytes, stream, nullptr,
+                          (unsigned long long)limit_us * 1000ull, 0);
 }
 
 sharq_status sharq_last_device_status(void* stream) {

@@ -147,18 +147,45 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and records a timeout)
-// when the phase does not complete within about a second.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// when the phase does not complete within limit_ns (about a second unless a
+// caller passes a shorter limit).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long t0 = globaltimer();
     while (true) {
         for (int i = 0; i < 8; ++i)
             if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             record_status(kStatusMbarTimeout);
             return false;
         }
     }
+}
+
+// Bounded grid-wide barrier for a cooperative launch (all blocks resident):
+// each block adds one arrival to *counter and waits until it reaches
+// target.  A wait that runs past limit_ns records a timeout and gives up,
+// so a lost block costs one limit per barrier instead of a hang.  skip: this
+// block does not arrive (only for the self-test of the timeout path).
+__device__ __forceinline__ void grid_barrier(uint32_t* counter, unsigned target,
+                                             unsigned long long limit_ns = kWaitLimitNs,
+                                             bool skip = false) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (!skip) atomicAdd(counter, 1u);
+        unsigned long long t0 = globaltimer();
+        while (ld_acquire_gpu(counter) < target) {
+            if (globaltimer() - t0 > limit_ns) {
+                record_status(kStatusGridTimeout);
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+    }
+    __syncthreads();
 }
 
 // ----------------------------------------------------------- clusters ----

@@ -13,17 +13,21 @@
 // warp owns whole rows, lane l reading the 16-byte chunks l, l+32, ... of a
 // row, which is also the fixed fp32 reduction order of the RMS sum; without
 // a norm, phase 1 is a plain maximum over the whole tensor, spread over every
-// lane.  Phases 2 and 3 spread (row, 256-element segment) items over every
-// warp.  MXFP4 has no tensor scale, so its backbone and residual are produced
-// in one pass (after the RMS barrier when there is a norm).  When the
-// producer of X has already taken A_b = max |X| (a no-norm input, e.g. the
-// SwiGLU epilogue of the gate+up linear), phase 1 and its barrier are
-// skipped: with the shared residual scale the whole prepare is then one
-// barrier-free pass.
+// lane.  Phases 2 and 3 give each lane whole scale blocks.  MXFP4 has no
+// tensor scale, so its backbone and residual are produced in one pass (after
+// the RMS barrier when there is a norm).  When the producer of X has already
+// taken A_b = max |X| (a no-norm input, e.g. the SwiGLU epilogue of the
+// gate+up linear), phase 1 and its barrier are skipped: with the shared
+// residual scale the whole prepare is then one barrier-free pass.
 //
-// Every floating-point step is one correctly rounded fp32 operation
-// (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn, no contraction), so the
+// Every floating-point step is one correctly rounded fp32 operation, so the
 // codes and scales are bit-identical to a plain sequential CPU evaluation.
+// The multiplications run as packed pairs (__fmul2_rn: per component the
+// same rounding as __fmul_rn) on the FMA pipe; additions and subtractions
+// stay scalar (a packed add after a packed multiply can be fused into one
+// rounding).  The integer and compare pipe, which bounds this kernel, is
+// kept for the mask, the maxima and the packing.  gamma (and beta) are converted to fp32
+// once per CTA into shared memory.
 #include "common.cuh"
 #include "sharq_internal.h"
 
@@ -39,6 +43,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// gamma / beta are staged in shared memory as fp32 up to this many bytes
+// (two CTAs per SM still fit); longer rows read them from global memory.
+constexpr int kMaxStagedBytes = 96 * 1024;
 
 struct PrepArgs {
     const uint16_t* X;       // [M, K] bf16
@@ -55,8 +62,14 @@ struct PrepArgs {
     uint8_t* rs_scales;
     float* rs_tscale;
     uint8_t* mask;           // optional
-    uint32_t* ws;            // [0] amax_b bits, [1] amax_r bits, [2] barrier, then rinv[M], mu[M]
+    uint32_t* ws;            // [0] amax_b bits, [1] amax_r bits, [2] barrier, [5] phase-2 guess
+                             // failed, [6] max pruned |y| bits; from word 16: rinv[M], mu[M]
     const float* amax_in;    // GIVEN: A_b = max |X| from the producer
+    int staged;              // gamma (and beta) are in shared memory as fp32
+    int spec;                // NVFP4 own residual scale: quantise the residual in phase 2 against
+                             // the largest pruned |y| (see phase 2)
+    unsigned long long wait_ns;   // limit of each grid-barrier wait
+    int skip_block;          // self-test only: this block never arrives at a barrier (-1: none)
 };
 
 __device__ __forceinline__ float* ws_rinv(uint32_t* ws) {
@@ -69,25 +82,34 @@ __device__ __forceinline__ int64_t sf_off(int64_t row, int s, int nsf) {
            ((row >> 5) & 3) * 4 + (s & 3);
 }
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float x[8]) {
-    x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-    x[4] = __uint_as_float(v.z << 16); x[5] = __uint_as_float(v.z & 0xFFFF0000u);
-    x[6] = __uint_as_float(v.w << 16); x[7] = __uint_as_float(v.w & 0xFFFF0000u);
+// Two bf16 (low half = first element) -> two exact fp32.
+__device__ __forceinline__ float2 bf16x2_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-// y = fl(fl(x * rinv) * gamma) for one chunk, or y = x without gamma.
-template <bool HAS_GAMMA>
-__device__ __forceinline__ void load_y(const PrepArgs& a, int64_t row, int c, float rinv,
-                                       float y[8]) {
-    uint4 v = ld_nc_v4(a.X + row * a.K + (int64_t)c * 8);
-    unpack_bf16x8(v, y);
-    if (HAS_GAMMA) {
-        float g[8];
-        unpack_bf16x8(ld_nc_v4(a.gamma + (int64_t)c * 8), g);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) y[t] = __fmul_rn(__fmul_rn(y[t], rinv), g[t]);
-    }
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float2 x[4]) {
+    x[0] = bf16x2_f2(v.x); x[1] = bf16x2_f2(v.y); x[2] = bf16x2_f2(v.z); x[3] = bf16x2_f2(v.w);
+}
+
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+
+// Packed pair multiply: per component one correctly rounded fp32 product,
+// the same bits as __fmul_rn.  There is no packed addition here on purpose:
+// a packed add that consumes a packed product may be fused with it into one
+// fused multiply-add (a single rounding) even when both are written with an
+// explicit rounding mode, which changes the residual's bits.  Every addition
+// and subtraction below is a scalar __fadd_rn / __fsub_rn, which is never
+// fused.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// fl(a - b) per component (scalar, never fused).
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) {
+    return make_float2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y));
+}
+
+// fl(a + b) per component (scalar, never fused).
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
 }
 
 // Top-n of every aligned group of MG inside the 8-element chunk; ties go to
@@ -113,16 +135,20 @@ __device__ __forceinline__ uint32_t topn_bits(const float y[8], int n) {
     return bits;
 }
 
-__device__ __forceinline__ float max3(float a, float b, float c) {
+__device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
 
-__device__ __forceinline__ float amax8(const float v[8]) {
-    float m0 = max3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
-    float m1 = max3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
-    return max3(m0, m1, fmaxf(fabsf(v[6]), fabsf(v[7])));
+// max |v| over N >= 3 values, three at a time.
+template <int N>
+__device__ __forceinline__ float amax_n(const float* v) {
+    float m = max3f(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+#pragma unroll
+    for (int i = 3; i + 1 < N; i += 2) m = max3f(m, fabsf(v[i]), fabsf(v[i + 1]));
+    if ((N - 3) % 2) m = fmaxf(m, fabsf(v[N - 1]));
+    return m;
 }
 
 // 2^p as fp32 for -127 <= p <= 127 (2^-127 is subnormal).
@@ -138,35 +164,60 @@ __device__ __forceinline__ uint32_t mx_code(float amax) {
     return (uint32_t)max(ef - 2, 0);
 }
 
-// Dequantised values of 8 packed codes: fl(fl(val * s) * g).  val * s is
-// exact in fp32; g is the decode tensor scale (1 for MXFP4).
-__device__ __forceinline__ void dequant8(uint32_t codes, float s, float g, float d[8]) {
+// Eight packed E2M1 codes -> four exact half2 pairs (element 2p low).
+__device__ __forceinline__ void e2m1x8_to_h2(uint32_t codes, __half2 h[4]) {
+    uint32_t r[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(codes));
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        uint32_t h2 = cvt_e2m1x2_to_f16x2((codes >> (8 * p)) & 0xFF);
-        float2 f = __half22float2(*reinterpret_cast<__half2*>(&h2));
-        d[2 * p] = __fmul_rn(__fmul_rn(f.x, s), g);
-        d[2 * p + 1] = __fmul_rn(__fmul_rn(f.y, s), g);
-    }
+    for (int p = 0; p < 4; ++p) h[p] = *reinterpret_cast<__half2*>(&r[p]);
 }
 
-// Bounded grid-wide barrier for a cooperative launch (all blocks resident).
-__device__ __forceinline__ void grid_barrier(uint32_t* counter, unsigned target) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(counter, 1u);
-        unsigned long long t0 = globaltimer();
-        while (ld_acquire_gpu(counter) < target) {
-            if (globaltimer() - t0 > kWaitLimitNs) {
-                record_status(kStatusGridTimeout);
-                break;
-            }
-            __nanosleep(64);
-        }
-        __threadfence();
-    }
-    __syncthreads();
+// An E4M3 scale code -> its exact value as f16 in both halves.
+__device__ __forceinline__ __half2 e4m3_h2(uint32_t code) {
+    uint32_t r;
+    const uint16_t two = (uint16_t)(code | (code << 8));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
+    return *reinterpret_cast<__half2*>(&r);
+}
+
+// Dequantised values of 8 packed NVFP4 codes: fl(fl(val * e) * G).  val * e
+// is exact in f16 (at least 0.5 * 2^-9 = 2^-10, a normal half, and at most
+// 6 * 448, with at most 6 significant bits), so the only rounding is that of
+// the multiplication by the tensor scale, as in the definition.
+__device__ __forceinline__ void dequant8_nv(uint32_t codes, __half2 e2, float2 g, float2 d[4]) {
+    __half2 h[4];
+    e2m1x8_to_h2(codes, h);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) d[p] = mul2_rn(__half22float2(__hmul2(h[p], e2)), g);
+}
+
+// Dequantised values of 8 packed MXFP4 codes: fl(val * 2^(c-127)).
+__device__ __forceinline__ void dequant8_mx(uint32_t codes, float2 sc, float2 d[4]) {
+    __half2 h[4];
+    e2m1x8_to_h2(codes, h);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) d[p] = mul2_rn(__half22float2(h[p]), sc);
+}
+
+// E2M1 codes of 8 values (pairs), element 2p in the low nibble of byte p.
+__device__ __forceinline__ uint32_t cvt_e2m1x8_f2(const float2 v[4]) {
+    return cvt_e2m1x8(reinterpret_cast<const float*>(v));
+}
+
+// Keep bits of 8 elements (bit t = element t) -> 0xF in nibble t: the AND
+// mask that clears the codes of pruned elements (code 0x0, +0).
+__device__ __forceinline__ uint32_t nibble_mask8(uint32_t k) {
+    uint32_t x = k & 0xFFu;
+    x = (x | (x << 12)) & 0x000F000Fu;
+    x = (x | (x << 6)) & 0x03030303u;
+    x = (x | (x << 3)) & 0x11111111u;
+    return x * 0xFu;
 }
 
 __device__ __forceinline__ void block_amax_to_global(float v, uint32_t* dst, float* red) {
@@ -214,21 +265,43 @@ __device__ __forceinline__ void fill_inv_table(float* tab, float genc) {
 
 // Walk the blocks b = start, start + stride, ... as (row, column) pairs
 // without a division per step.
+// Work distribution of phases 2 and 3 over the flattened [M, K/E] scale
+// blocks: lane l of global warp w starts at block 32w + l and steps by the
+// number of lanes in the grid, so a warp's 32 blocks are always 32 * E
+// consecutive elements (coalesced loads, one 8- or 16-byte code store per
+// lane).  REV walks the same sequence from the far end of X: phase 2 starts
+// on the rows phase 1 read last, which are still in L2 when X is larger
+// than L2, and phase 3 (forwards) starts on the rows phase 2 read last.
+// (Measured alternatives, slower: each warp taking runs of 512 consecutive
+// blocks, and runs handed out from one atomic counter -- one counter
+// serialises at about 10^8 atomics per second.)
+template <bool REV>
 struct BlockCursor {
-    int64_t row;
-    int cb;
-    int dr, dc, nbr;
-    __device__ __forceinline__ void init(int64_t start, int64_t stride, int nb_row) {
-        nbr = nb_row;
-        row = start / nb_row;
-        cb = (int)(start - row * nb_row);
-        dr = (int)(stride / nb_row);
-        dc = (int)(stride - (int64_t)dr * nb_row);
+    int64_t row;           // this lane's block (only meaningful while valid())
+    int cb, nbr, dr, dc;
+    int i;                 // steps taken (the same in every lane)
+    int64_t sfo;           // byte offset of the block's scale, sf_off(row, cb, nbr)
+    int64_t wpos, wstride, total, nrows;
+    __device__ __forceinline__ void init(int64_t gw, int64_t nw, int64_t tot, int nb_row, int lane) {
+        nbr = nb_row; i = 0; total = tot; nrows = tot / nb_row;
+        wpos = gw * 32;                       // lane 0's position in the walk
+        wstride = nw * 32;
+        const int64_t j = wpos + lane;
+        const int64_t b = REV ? tot - 1 - j : j;
+        row = b >= 0 ? b / nb_row : -1;
+        cb = (int)(b - row * nb_row);
+        dr = (int)(wstride / nb_row);
+        dc = (int)(wstride - (int64_t)dr * nb_row);
+        sfo = sf_off(row, cb, nb_row);
     }
+    __device__ __forceinline__ bool live() const { return wpos < total; }   // the same in every lane
+    __device__ __forceinline__ bool valid() const { return row >= 0 && row < nrows; }
     __device__ __forceinline__ void next() {
-        cb += dc;
-        row += dr;
-        if (cb >= nbr) { cb -= nbr; ++row; }
+        ++i;
+        wpos += wstride;
+        if (REV) { cb -= dc; row -= dr; if (cb < 0) { cb += nbr; --row; } }
+        else     { cb += dc; row += dr; if (cb >= nbr) { cb -= nbr; ++row; } }
+        sfo = sf_off(row, cb, nbr);
     }
 };
 
@@ -257,12 +330,96 @@ __device__ __forceinline__ uint32_t keep_bits(const float* y, int n) {
     return k;
 }
 
-template <int E>
-__device__ __forceinline__ float amaxE(const float* v) {
-    float m = amax8(v);
+template <uint32_t LUT>
+__device__ __forceinline__ uint32_t lop3t(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(a), "r"(b), "r"(c), "n"(LUT));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// The 2-of-4 mask of 8 elements as the AND mask of their packed codes (0xF
+// in nibble t when element t is kept).  Each comparison |a| >= |b| is the
+// sign of the exact difference fl(|a| - |b|) (no rounding can turn a
+// nonzero difference into zero or flip its sign; equal magnitudes give +0),
+// taken on the FMA pipe; the four keep decisions of a group are majority
+// functions of three such signs, one lop3 each (element i is kept when it
+// beats at least two of the other three; a tie goes to the lower index):
+//   k0 = maj(a0>=a1, a0>=a2, a0>=a3)   k1 = maj(a1>a0, a1>=a2, a1>=a3)
+//   k2 = maj(a2>a0, a2>a1, a2>=a3)     k3 = maj(a3>a0, a3>a1, a3>a2).
+// The keep bit is bit 31 of k_i; byte permutes with sign replication turn
+// those bits into byte masks, and one lop3 merges the even and odd elements
+// into nibbles.
+__device__ __forceinline__ uint32_t keep24_nibbles8(const float* y) {
+    uint32_t k[8];
 #pragma unroll
-    for (int g = 8; g < E; g += 8) m = fmaxf(m, amax8(v + g));
+    for (int g = 0; g < 8; g += 4) {
+        const float a0 = fabsf(y[g]), a1 = fabsf(y[g + 1]), a2 = fabsf(y[g + 2]), a3 = fabsf(y[g + 3]);
+        const uint32_t d01 = __float_as_uint(__fsub_rn(a0, a1)), d02 = __float_as_uint(__fsub_rn(a0, a2));
+        const uint32_t d03 = __float_as_uint(__fsub_rn(a0, a3)), d12 = __float_as_uint(__fsub_rn(a1, a2));
+        const uint32_t d13 = __float_as_uint(__fsub_rn(a1, a3)), d23 = __float_as_uint(__fsub_rn(a2, a3));
+        // sign bit set = the first operand is smaller
+        k[g] = lop3t<0x17>(d01, d02, d03);        // maj(~s01, ~s02, ~s03)
+        k[g + 1] = lop3t<0x71>(d01, d12, d13);    // maj(s01, ~s12, ~s13)
+        k[g + 2] = lop3t<0xD4>(d02, d12, d23);    // maj(s02, s12, ~s23)
+        k[g + 3] = lop3t<0xE8>(d03, d13, d23);    // maj(s03, s13, s23)
+    }
+    // sign-replicated byte 3 of each word: 0xFF when kept
+    const uint32_t e01 = prmt(k[0], k[2], 0x00FBu), e23 = prmt(k[4], k[6], 0xFB00u);
+    const uint32_t o01 = prmt(k[1], k[3], 0x00FBu), o23 = prmt(k[5], k[7], 0xFB00u);
+    const uint32_t ev = prmt(e01, e23, 0x7610u), od = prmt(o01, o23, 0x7610u);
+    return lop3t<0xE4>(ev, od, 0x0F0F0F0Fu);      // (ev & 0x0F..) | (od & 0xF0..)
+}
+
+// Keep bits (bit t = element t) of a code AND mask (0xF in nibble t).
+__device__ __forceinline__ uint32_t nibbles_to_bits8(uint32_t m) {
+    uint32_t b = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) b |= ((m >> (4 * t)) & 1u) << t;
+    return b;
+}
+
+// The second smallest of four magnitudes: the larger of the two pruned ones
+// under the 2-of-4 mask (ties prune equal values, so the value is the same
+// whichever index is pruned).
+__device__ __forceinline__ float second_smallest4(const float* y) {
+    const float a = fabsf(y[0]), b = fabsf(y[1]), c = fabsf(y[2]), d = fabsf(y[3]);
+    return fminf(fmaxf(fminf(a, b), fminf(c, d)), fminf(fmaxf(a, b), fmaxf(c, d)));
+}
+
+// max |y| over the entries of an aligned 8-element chunk that the mask prunes.
+template <int MG, bool NM24>
+__device__ __forceinline__ float pruned_max8(const float* y, int n) {
+    if (NM24) return fmaxf(second_smallest4(y), second_smallest4(y + 4));
+    const uint32_t k = keep_bits<8, MG, NM24>(y, n);
+    float m = 0.0f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m = fmaxf(m, ((k >> t) & 1u) ? 0.0f : fabsf(y[t]));
     return m;
+}
+
+// gamma / beta of elements [c0, c0 + 2P) as fp32 pairs: from the shared
+// fp32 copy, or converted from global bf16.
+template <int P>
+__device__ __forceinline__ void load_vec2(const float* sv, const uint16_t* gv, bool staged, int c0,
+                                          float2 out[P]) {
+    if (staged) {
+        const float4* s4 = reinterpret_cast<const float4*>(sv + c0);
+#pragma unroll
+        for (int p = 0; p < P; p += 2) {
+            const float4 v = s4[p / 2];
+            out[p] = make_float2(v.x, v.y);
+            out[p + 1] = make_float2(v.z, v.w);
+        }
+    } else {
+#pragma unroll
+        for (int p = 0; p < P; p += 4) unpack_bf16x8(ld_nc_v4(gv + c0 + 2 * p), out + p);
+    }
 }
 
 template <int FMT, bool HAS_GAMMA, bool LN>
@@ -270,48 +427,36 @@ struct LaneBlock {
     static constexpr int E = FMT == 0 ? 16 : 32;   // elements per lane = one scale block
     static constexpr int NV = E / 8;                // 16-byte chunks
     uint4 x[NV];
-    uint4 g[NV];
-    uint4 b[LN ? NV : 1];
     float rinv, mu;
 
     __device__ __forceinline__ void load(const PrepArgs& a, int64_t row, int cb, const float* rinv_ws) {
         const uint16_t* xp = a.X + row * a.K + (int64_t)cb * E;
 #pragma unroll
         for (int v = 0; v < NV; ++v) x[v] = ld_nc_v4(xp + 8 * v);
-        if (HAS_GAMMA) {
-#pragma unroll
-            for (int v = 0; v < NV; ++v) g[v] = ld_nc_v4(a.gamma + (int64_t)cb * E + 8 * v);
-            rinv = rinv_ws[row];
-        }
-        if (LN) {
-            mu = rinv_ws[a.M + row];          // the LayerNorm means follow the M reciprocals
-            if (a.beta) {
-#pragma unroll
-                for (int v = 0; v < NV; ++v) b[v] = ld_nc_v4(a.beta + (int64_t)cb * E + 8 * v);
-            }
-        }
+        if (HAS_GAMMA) rinv = rinv_ws[row];
+        if (LN) mu = rinv_ws[a.M + row];          // the LayerNorm means follow the M reciprocals
     }
 
     // RMSNorm: fl(fl(x * rinv) * g).  LayerNorm: fl(fl(fl(x - mu) * rstd) * g),
-    // then + beta when there is a bias.
-    __device__ __forceinline__ void y(float* out, bool has_beta) const {
+    // then + beta when there is a bias.  Without a norm y = x.
+    __device__ __forceinline__ void y(float2* out, int cb, const PrepArgs& a, const float* sg,
+                                      const float* sb, bool has_beta) const {
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            unpack_bf16x8(x[v], out + 8 * v);
-            if (HAS_GAMMA) {
-                float gg[8];
-                unpack_bf16x8(g[v], gg);
+        for (int v = 0; v < NV; ++v) unpack_bf16x8(x[v], out + 4 * v);
+        if (HAS_GAMMA) {
+            float2 g[E / 2];
+            load_vec2<E / 2>(sg, a.gamma, a.staged, cb * E, g);
+            const float2 r2 = f2(rinv), mu2 = f2(mu);
 #pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const float xv = LN ? __fsub_rn(out[8 * v + t], mu) : out[8 * v + t];
-                    out[8 * v + t] = __fmul_rn(__fmul_rn(xv, rinv), gg[t]);
-                }
-                if (LN && has_beta) {
-                    float bb[8];
-                    unpack_bf16x8(b[v], bb);
+            for (int p = 0; p < E / 2; ++p) {
+                float2 t = LN ? sub2_rn(out[p], mu2) : out[p];
+                out[p] = mul2_rn(mul2_rn(t, r2), g[p]);
+            }
+            if (LN && has_beta) {
+                float2 b[E / 2];
+                load_vec2<E / 2>(sb, a.beta, a.staged, cb * E, b);
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) out[8 * v + t] = __fadd_rn(out[8 * v + t], bb[t]);
-                }
+                for (int p = 0; p < E / 2; ++p) out[p] = add2_rn(out[p], b[p]);
             }
         }
     }
@@ -328,7 +473,10 @@ template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS, bool
 __global__ void __launch_bounds__(kThreads, 2)
 prepare_kernel(PrepArgs a) {
     __shared__ float s_inv[128];
+    __shared__ float s_inv_p[128];    // SPEC: reciprocal table of the residual's guessed scale
     __shared__ float s_red[kWarps];
+    __shared__ unsigned s_spec_sent;  // SPEC: this CTA has met a residual block above P
+    extern __shared__ __align__(16) float s_vec[];     // gamma [K] (then beta [K]) as fp32
     using LB = LaneBlock<FMT, HAS_GAMMA, LN>;
     static_assert(!LN || HAS_GAMMA, "LayerNorm takes gamma");
     static_assert(!GIVEN || (FMT == 0 && !HAS_GAMMA && !WEIGHT), "a given amax: NVFP4, no norm");
@@ -345,9 +493,31 @@ prepare_kernel(PrepArgs a) {
     const int64_t M = a.M;
     const int64_t Mpad = (M + 127) / 128 * 128;
     float* rinv_ws = ws_rinv(a.ws);
+    const bool skip = (int)blockIdx.x == a.skip_block;
+    // NVFP4 with its own residual scale: phase 1 also takes P = max |y| over
+    // the pruned entries, and phase 2 quantises the residual against P (see
+    // the end of phase 2).
+    constexpr bool SPEC = FMT == 0 && !WEIGHT && !RS && !GIVEN;
+    const bool spec = SPEC && a.spec;
+    float* s_gamma = s_vec;
+    float* s_beta = s_vec + K;
+    if (threadIdx.x == 0) s_spec_sent = 0u;    // read only after phase 1's block reductions
+
+    if (HAS_GAMMA && a.staged) {
+        for (int i = threadIdx.x; i < K / 2; i += kThreads) {
+            const float2 g = bf16x2_f2(reinterpret_cast<const uint32_t*>(a.gamma)[i]);
+            s_gamma[2 * i] = g.x; s_gamma[2 * i + 1] = g.y;
+            if (has_beta) {
+                const float2 b = bf16x2_f2(reinterpret_cast<const uint32_t*>(a.beta)[i]);
+                s_beta[2 * i] = b.x; s_beta[2 * i + 1] = b.y;
+            }
+        }
+        __syncthreads();
+    }
 
     // ---------------- phase 1: rinv per row, A_b = max |y| ----------------
     float amax = 0.0f;
+    float pmax = 0.0f;     // SPEC: max |y| over the pruned entries
     if (FMT == 0 && !HAS_GAMMA && !GIVEN) {
         // y = x, and A_b = max |x| needs no row structure: lane i of the
         // grid reads chunks i, i + L, ..., i + 15L (L = lanes in the grid),
@@ -369,6 +539,13 @@ prepare_kernel(PrepArgs a) {
                     m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
                     m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
                     m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+                    if (spec) {
+                        // chunks start at multiples of 8 elements, so the
+                        // mask's aligned groups lie inside one chunk
+                        float2 x2[4];
+                        unpack_bf16x8(v[u], x2);
+                        pmax = fmaxf(pmax, pruned_max8<MG, NM24>(reinterpret_cast<const float*>(x2), a.n));
+                    }
                 }
             }
         }
@@ -377,7 +554,7 @@ prepare_kernel(PrepArgs a) {
         // One warp per row.  rinv: lane l adds f(x) over chunks l, l+32, ...
         // element by element in k order, then the xor butterfly -- the fixed
         // reduction order.  Then (NVFP4) the row's max |y|.  Eight chunk
-        // loads in flight per lane (four per operand for LayerNorm's max).
+        // loads in flight per lane.
         for (int64_t row = gwarp; row < M; row += nwarps) {
             const uint16_t* xr = a.X + row * K;
             auto row_sum = [&](auto f) {
@@ -390,10 +567,13 @@ prepare_kernel(PrepArgs a) {
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         if (c0 + 32 * u < nchunk) {
-                            float x[8];
+                            float2 x[4];
                             unpack_bf16x8(v[u], x);
 #pragma unroll
-                            for (int t = 0; t < 8; ++t) acc = __fadd_rn(acc, f(x[t]));
+                            for (int t = 0; t < 4; ++t) {
+                                acc = __fadd_rn(acc, f(x[t].x));
+                                acc = __fadd_rn(acc, f(x[t].y));
+                            }
                         }
                     }
                 }
@@ -418,35 +598,33 @@ prepare_kernel(PrepArgs a) {
                 if (lane == 0) rinv_ws[row] = rinv;
             }
             if (FMT == 0) {
-                constexpr int D = LN ? 4 : 8;   // LayerNorm also streams beta
+                const float2 r2 = f2(rinv), mu2 = f2(mu);
+                constexpr int D = LN ? 4 : 8;   // LayerNorm also reads beta
                 for (int c0 = lane; c0 < nchunk; c0 += 32 * D) {
-                    uint4 v[D], g[D], bt[LN ? D : 1];
+                    uint4 v[D];
+#pragma unroll
+                    for (int u = 0; u < D; ++u)
+                        if (c0 + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
 #pragma unroll
                     for (int u = 0; u < D; ++u) {
                         if (c0 + 32 * u < nchunk) {
-                            v[u] = ld_nc_v4(xr + (int64_t)(c0 + 32 * u) * 8);
-                            g[u] = ld_nc_v4(a.gamma + (int64_t)(c0 + 32 * u) * 8);
-                            if (LN && has_beta) bt[u] = ld_nc_v4(a.beta + (int64_t)(c0 + 32 * u) * 8);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < D; ++u) {
-                        if (c0 + 32 * u < nchunk) {
-                            float y[8], gg[8];
+                            const int c = c0 + 32 * u;
+                            float2 y[4], g[4];
                             unpack_bf16x8(v[u], y);
-                            unpack_bf16x8(g[u], gg);
+                            load_vec2<4>(s_gamma, a.gamma, a.staged, c * 8, g);
 #pragma unroll
-                            for (int t = 0; t < 8; ++t) {
-                                const float xv = LN ? __fsub_rn(y[t], mu) : y[t];
-                                y[t] = __fmul_rn(__fmul_rn(xv, rinv), gg[t]);
+                            for (int t = 0; t < 4; ++t) {
+                                const float2 xv = LN ? sub2_rn(y[t], mu2) : y[t];
+                                y[t] = mul2_rn(mul2_rn(xv, r2), g[t]);
                             }
                             if (LN && has_beta) {
-                                float bb[8];
-                                unpack_bf16x8(bt[u], bb);
+                                float2 b[4];
+                                load_vec2<4>(s_beta, a.beta, a.staged, c * 8, b);
 #pragma unroll
-                                for (int t = 0; t < 8; ++t) y[t] = __fadd_rn(y[t], bb[t]);
+                                for (int t = 0; t < 4; ++t) y[t] = add2_rn(y[t], b[t]);
                             }
-                            amax = fmaxf(amax, amax8(y));
+                            amax = fmaxf(amax, amax_n<8>(reinterpret_cast<const float*>(y)));
+                            if (spec) pmax = fmaxf(pmax, pruned_max8<MG, NM24>(reinterpret_cast<const float*>(y), a.n));
                         }
                     }
                 }
@@ -456,9 +634,10 @@ prepare_kernel(PrepArgs a) {
 
     if (FMT == 0 && !GIVEN) {
         block_amax_to_global(amax, &a.ws[0], s_red);
-        grid_barrier(&a.ws[2], gridDim.x);
+        if (spec) block_amax_to_global(pmax, &a.ws[6], s_red);
+        grid_barrier(&a.ws[2], gridDim.x, a.wait_ns, skip);
     } else if (HAS_GAMMA) {
-        grid_barrier(&a.ws[2], gridDim.x);   // rinv of every row visible to every warp
+        grid_barrier(&a.ws[2], gridDim.x, a.wait_ns, skip);   // rinv of every row visible to every warp
     }
 
     // ------- phase 2: mask, backbone, residual amax (and MXFP4 residual) -------
@@ -490,176 +669,254 @@ prepare_kernel(PrepArgs a) {
     }
 
     const int nb_row = K / E;
+    const float2 gb2 = f2(sb.gdec);
+    NvScale sp{1.0f, 1.0f, 1.0f};
+    uint32_t pbits = 0;
+    if (spec) {
+        pbits = ld_acquire_gpu(&a.ws[6]);
+        sp = nv_scale(__uint_as_float(pbits));
+        fill_inv_table(s_inv_p, sp.genc);
+        if (blockIdx.x == 0 && threadIdx.x == 0) *a.rs_tscale = sp.gdec;
+    }
+    const bool guess = spec;
+    bool spec_on = guess;      // this lane still writes residual codes against P
     float ramax = 0.0f;
     {
-        BlockCursor cur;
-        cur.init(gwarp * 32 + lane, nwarps * 32, nb_row);
+        BlockCursor<true> cur;
+        cur.init(gwarp, nwarps, M * nb_row, nb_row, lane);
         LB lb;
-        if (cur.row < M) lb.load(a, cur.row, cur.cb, rinv_ws);
-        while (cur.row < M) {
-            BlockCursor nxt = cur;
+        if (cur.live() && cur.valid()) lb.load(a, cur.row, cur.cb, rinv_ws);
+        while (cur.live()) {
+            if (guess && (cur.i & 3) == 0) {
+                // Once any lane anywhere has met a residual block above P the
+                // guess is wrong and phase 3 will run: stop writing residual
+                // codes.  One global flag write per CTA; each warp reads the
+                // flag every fourth block, each lane its CTA's flag every block.
+                uint32_t f = 0;
+                if (lane == 0) f = ld_acquire_gpu(&a.ws[5]);
+                if (__shfl_sync(0xffffffffu, f, 0)) spec_on = false;
+            }
+            if (spec_on && *reinterpret_cast<volatile unsigned*>(&s_spec_sent)) spec_on = false;
+            BlockCursor<true> nxt = cur;
             nxt.next();
             LB ln;
-            if (nxt.row < M) ln.load(a, nxt.row, nxt.cb, rinv_ws);   // prefetch
-
+            if (nxt.live() && nxt.valid()) ln.load(a, nxt.row, nxt.cb, rinv_ws);   // prefetch
+            if (cur.valid()) {
             const int64_t row = cur.row;
             const int cb = cur.cb;
-            float y[E];
-            lb.y(y, has_beta);
+            float2 y2[E / 2];
+            lb.y(y2, cb, a, s_gamma, s_beta, has_beta);
+            const float* y = reinterpret_cast<const float*>(y2);
             // the backbone's block max is the block max of y: the largest
             // entry of every group is always kept
-            const float bm = amaxE<E>(y);
+            const float bm = amax_n<E>(y);
             uint32_t ecode;
-            float inv, sdec;
+            float inv;
             if (FMT == 0) {
                 ecode = cvt_e4m3(__fmul_rn(bm, sb.k1));
                 inv = s_inv[ecode];
-                sdec = e4m3_to_f32(ecode);
             } else {
                 ecode = mx_code(bm);
                 inv = pow2f(127 - (int)ecode);
-                sdec = pow2f((int)ecode - 127);
             }
-            const uint32_t keep = WEIGHT ? 0xFFFFFFFFu : keep_bits<E, MG, NM24>(y, a.n);
-            uint32_t codes[E / 8];
+            // the mask as one code AND mask (0xF per kept element) per 8 elements
+            uint32_t kmask[E / 8];
 #pragma unroll
             for (int v = 0; v < E / 8; ++v) {
-                float t8[8];
+                if (WEIGHT)     kmask[v] = 0xFFFFFFFFu;
+                else if (NM24)  kmask[v] = keep24_nibbles8(y + 8 * v);
+                else            kmask[v] = nibble_mask8(keep_bits<8, MG, NM24>(y + 8 * v, a.n));
+            }
+            uint32_t codes[E / 8];
+            const float2 inv2 = f2(inv);
 #pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    t8[t] = ((keep >> (8 * v + t)) & 1u) ? __fmul_rn(y[8 * v + t], inv) : 0.0f;
-                codes[v] = cvt_e2m1x8(t8);
+            for (int v = 0; v < E / 8; ++v) {
+                float2 q[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[4 * v + p], inv2);
+                codes[v] = cvt_e2m1x8_f2(q) & kmask[v];   // pruned: code 0 (+0)
             }
             uint8_t* cp = a.bb_codes + row * (K / 2) + (int64_t)cb * (E / 2);
             if (E == 16) *reinterpret_cast<uint2*>(cp) = make_uint2(codes[0], codes[1]);
             else         *reinterpret_cast<uint4*>(cp) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            a.bb_scales[sf_off(row, cb, nsf)] = (uint8_t)ecode;
+            a.bb_scales[cur.sfo] = (uint8_t)ecode;
             if (!WEIGHT && a.mask) {
                 uint8_t* mp = a.mask + row * (K / 8) + (int64_t)cb * (E / 8);
-                if (E == 16) *reinterpret_cast<uint16_t*>(mp) = (uint16_t)keep;
-                else         *reinterpret_cast<uint32_t*>(mp) = keep;
+#pragma unroll
+                for (int v = 0; v < E / 8; ++v) mp[v] = (uint8_t)nibbles_to_bits8(kmask[v]);
             }
 
             if (!WEIGHT) {
-                // residual r = y - dequant(backbone), in place in y
+                // residual r = y - dequant(backbone), in place in y2
+                const __half2 eh = e4m3_h2(FMT == 0 ? ecode : 0u);
+                const float2 sd2 = f2(pow2f((int)ecode - 127));
 #pragma unroll
                 for (int v = 0; v < E / 8; ++v) {
-                    float d[8];
-                    dequant8(codes[v], sdec, sb.gdec, d);
+                    float2 d[4];
+                    if (FMT == 0) dequant8_nv(codes[v], eh, gb2, d);
+                    else          dequant8_mx(codes[v], sd2, d);
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) y[8 * v + t] = __fsub_rn(y[8 * v + t], d[t]);
+                    for (int p = 0; p < 4; ++p) y2[4 * v + p] = sub2_rn(y2[4 * v + p], d[p]);
                 }
+                const float rbm = amax_n<E>(y);
                 if (FMT == 0 && RS) {
                     // the residual's block scale against the backbone's G
-                    const uint32_t er = cvt_e4m3(__fmul_rn(amaxE<E>(y), sb.k1));
-                    const float inv_r = s_inv[er];
+                    const uint32_t er = cvt_e4m3(__fmul_rn(rbm, sb.k1));
+                    const float2 ir2 = f2(s_inv[er]);
                     uint32_t rc[E / 8];
 #pragma unroll
                     for (int v = 0; v < E / 8; ++v) {
-                        float t8[8];
+                        float2 q[4];
 #pragma unroll
-                        for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[8 * v + t], inv_r);
-                        rc[v] = cvt_e2m1x8(t8);
+                        for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[4 * v + p], ir2);
+                        rc[v] = cvt_e2m1x8_f2(q);
                     }
                     *reinterpret_cast<uint2*>(a.rs_codes + row * (K / 2) + (int64_t)cb * 8) = make_uint2(rc[0], rc[1]);
-                    a.rs_scales[sf_off(row, cb, nsf)] = (uint8_t)er;
+                    a.rs_scales[cur.sfo] = (uint8_t)er;
                 } else if (FMT == 0) {
-                    ramax = fmaxf(ramax, amaxE<E>(y));
+                    ramax = fmaxf(ramax, rbm);
+                    if (spec_on) {
+                        if (__float_as_uint(rbm) > pbits) {   // A_r > P: phase 3 will run
+                            if (atomicExch(&s_spec_sent, 1u) == 0u) atomicOr(&a.ws[5], 1u);
+                            spec_on = false;
+                        } else {
+                            const uint32_t er = cvt_e4m3(__fmul_rn(rbm, sp.k1));
+                            const float2 ir2 = f2(s_inv_p[er]);
+                            uint32_t rc[2];
+#pragma unroll
+                            for (int v = 0; v < 2; ++v) {
+                                float2 q[4];
+#pragma unroll
+                                for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[4 * v + p], ir2);
+                                rc[v] = cvt_e2m1x8_f2(q);
+                            }
+                            *reinterpret_cast<uint2*>(a.rs_codes + row * (K / 2) + (int64_t)cb * 8) = make_uint2(rc[0], rc[1]);
+                            a.rs_scales[cur.sfo] = (uint8_t)er;
+                        }
+                    }
                 } else {
                     // MXFP4: the residual needs no tensor-wide scale; finish it here.
-                    const uint32_t rcode = mx_code(amaxE<E>(y));
-                    const float rs = pow2f(127 - (int)rcode);
+                    const uint32_t rcode = mx_code(rbm);
+                    const float2 rs2 = f2(pow2f(127 - (int)rcode));
                     uint32_t rc[E / 8];
 #pragma unroll
                     for (int v = 0; v < E / 8; ++v) {
-                        float t8[8];
+                        float2 q[4];
 #pragma unroll
-                        for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[8 * v + t], rs);
-                        rc[v] = cvt_e2m1x8(t8);
+                        for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[4 * v + p], rs2);
+                        rc[v] = cvt_e2m1x8_f2(q);
                     }
                     *reinterpret_cast<uint4*>(a.rs_codes + row * (K / 2) + (int64_t)cb * (E / 2)) =
                         make_uint4(rc[0], rc[1], rc[2], rc[3]);
-                    a.rs_scales[sf_off(row, cb, nsf)] = (uint8_t)rcode;
+                    a.rs_scales[cur.sfo] = (uint8_t)rcode;
                 }
             }
+            }   // valid
             cur = nxt;
             lb = ln;
         }
     }
-    if (FMT == 1 || WEIGHT || RS) return;
+    if constexpr (FMT == 0 && !WEIGHT && !RS) {
 
     block_amax_to_global(ramax, &a.ws[1], s_red);
-    grid_barrier(&a.ws[2], (GIVEN ? 1u : 2u) * gridDim.x);   // counts on from phase 1's
+    grid_barrier(&a.ws[2], (GIVEN ? 1u : 2u) * gridDim.x, a.wait_ns, skip);   // counts on from phase 1's
 
+    // The residual's tensor max is A_r = max(P, Q): P = max |y| over the
+    // pruned entries (whose residual is y itself) and Q = max |y - D_b| over
+    // the kept ones.  Phase 1 took P; phase 2, which is the first to know Q,
+    // already quantised every residual block against P.  When A_r == P those
+    // codes, scales and G_r are the final ones and phase 3 is not needed.
+    const uint32_t arbits = ld_acquire_gpu(&a.ws[1]);
+    if (guess && arbits == pbits) return;
     // ---------------- phase 3: residual codes with G_r ----------------
-    NvScale sr = nv_scale(__uint_as_float(ld_acquire_gpu(&a.ws[1])));
+    NvScale sr = nv_scale(__uint_as_float(arbits));
     __syncthreads();                       // everyone done reading the backbone table
     fill_inv_table(s_inv, sr.genc);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.rs_tscale = sr.gdec;
     {
-        BlockCursor cur;
-        cur.init(gwarp * 32 + lane, nwarps * 32, nb_row);
+        BlockCursor<false> cur;
+        cur.init(gwarp, nwarps, M * nb_row, nb_row, lane);
         LB lb;
         uint2 bc = make_uint2(0, 0);
         uint32_t bs = 0;
-        if (cur.row < M) {
+        if (cur.live() && cur.valid()) {
             lb.load(a, cur.row, cur.cb, rinv_ws);
             bc = *reinterpret_cast<const uint2*>(a.bb_codes + cur.row * (K / 2) + (int64_t)cur.cb * 8);
-            bs = a.bb_scales[sf_off(cur.row, cur.cb, nsf)];
+            bs = a.bb_scales[cur.sfo];
         }
-        while (cur.row < M) {
-            BlockCursor nxt = cur;
+        while (cur.live()) {
+            BlockCursor<false> nxt = cur;
             nxt.next();
             LB ln;
             uint2 nbc = make_uint2(0, 0);
             uint32_t nbs = 0;
-            if (nxt.row < M) {
+            if (nxt.live() && nxt.valid()) {
                 ln.load(a, nxt.row, nxt.cb, rinv_ws);
                 nbc = *reinterpret_cast<const uint2*>(a.bb_codes + nxt.row * (K / 2) + (int64_t)nxt.cb * 8);
-                nbs = a.bb_scales[sf_off(nxt.row, nxt.cb, nsf)];
+                nbs = a.bb_scales[nxt.sfo];
             }
+            if (cur.valid()) {
             const int64_t row = cur.row;
             const int cb = cur.cb;
-            float y[16];
-            lb.y(y, has_beta);
-            const float sdec = e4m3_to_f32(bs);
-            float d[8];
-            dequant8(bc.x, sdec, sb.gdec, d);
+            float2 y2[8];
+            lb.y(y2, cb, a, s_gamma, s_beta, has_beta);
+            const __half2 eh = e4m3_h2(bs);
+            float2 d[4];
+            dequant8_nv(bc.x, eh, gb2, d);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) y[t] = __fsub_rn(y[t], d[t]);
-            dequant8(bc.y, sdec, sb.gdec, d);
+            for (int p = 0; p < 4; ++p) y2[p] = sub2_rn(y2[p], d[p]);
+            dequant8_nv(bc.y, eh, gb2, d);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) y[8 + t] = __fsub_rn(y[8 + t], d[t]);   // y := r
-            const uint32_t er = cvt_e4m3(__fmul_rn(amaxE<16>(y), sr.k1));
-            const float inv = s_inv[er];
-            float t8[8];
+            for (int p = 0; p < 4; ++p) y2[4 + p] = sub2_rn(y2[4 + p], d[p]);   // y2 := r
+            const uint32_t er = cvt_e4m3(__fmul_rn(amax_n<16>(reinterpret_cast<const float*>(y2)), sr.k1));
+            const float2 inv2 = f2(s_inv[er]);
+            float2 q[4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[t], inv);
-            const uint32_t c0 = cvt_e2m1x8(t8);
+            for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[p], inv2);
+            const uint32_t c0 = cvt_e2m1x8_f2(q);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) t8[t] = __fmul_rn(y[8 + t], inv);
-            const uint32_t c1 = cvt_e2m1x8(t8);
+            for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[4 + p], inv2);
+            const uint32_t c1 = cvt_e2m1x8_f2(q);
             *reinterpret_cast<uint2*>(a.rs_codes + row * (K / 2) + (int64_t)cb * 8) = make_uint2(c0, c1);
-            a.rs_scales[sf_off(row, cb, nsf)] = (uint8_t)er;
+            a.rs_scales[cur.sfo] = (uint8_t)er;
+            }   // valid
             cur = nxt;
             lb = ln;
             bc = nbc;
             bs = nbs;
         }
     }
+    }   // phase 3
 }
 
 template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false, bool LN = false,
           bool GIVEN = false>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN, GIVEN>;
-    // same for every device of one architecture; a repeated query is harmless
-    static std::atomic<int> cached{0};
-    int blocks_per_sm = cached.load(std::memory_order_relaxed);
+    const size_t smem = a.staged ? (size_t)a.K * 4 * (LN && a.beta ? 2 : 1) : 0;
+    // Resident blocks per SM at this shared-memory size (the cooperative
+    // grid must not exceed it); the same for every device of one
+    // architecture, so cache the answer per size class.
+    static std::atomic<int> cached[4];
+    const int cls = smem == 0 ? 0 : smem <= 32 * 1024 ? 1 : smem <= 64 * 1024 ? 2 : 3;
+    const size_t cls_bytes[4] = {0, 32 * 1024, 64 * 1024, (size_t)kMaxStagedBytes};
+    int blocks_per_sm = cached[cls].load(std::memory_order_relaxed);
     if (blocks_per_sm == 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kfn, kThreads, 0);
+        if (cls_bytes[cls] > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kMaxStagedBytes);
+            if (e != cudaSuccess) return e;
+        }
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kfn, kThreads,
+                                                                      cls_bytes[cls]);
         if (e != cudaSuccess) return e;
-        cached.store(blocks_per_sm, std::memory_order_relaxed);
+        if (blocks_per_sm < 1) return cudaErrorInvalidConfiguration;
+        cached[cls].store(blocks_per_sm, std::memory_order_relaxed);
+    }
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kMaxStagedBytes);
+        if (e != cudaSuccess) return e;
     }
     // Enough warps for one row each in phase 1 and about four 32-block
     // groups each in phases 2 and 3, capped at what is resident.
@@ -667,11 +924,11 @@ cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
     int64_t groups = a.M * (int64_t)(a.K / (FMT == 0 ? 16 : 32)) / 32;
     int64_t want = std::max((Mpad + kWarps - 1) / kWarps, (groups + 4 * kWarps - 1) / (4 * kWarps));
     int64_t cap = (int64_t)blocks_per_sm * max_blocks;
-    int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
+    int grid = (int)std::max<int64_t>(1, std::min(want, cap));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;   // grid barriers: all blocks co-resident
@@ -720,6 +977,11 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     a.ws = static_cast<uint32_t*>(p.ws);
     a.amax_in = p.amax;
     const bool g = p.gamma != nullptr;
+    const size_t vec_bytes = (size_t)p.K * 4 * (p.layernorm && p.beta ? 2 : 1);
+    a.staged = g && vec_bytes <= (size_t)kMaxStagedBytes;
+    a.spec = p.spec_off ? 0 : 1;
+    a.wait_ns = p.wait_ns ? p.wait_ns : kWaitLimitNs;
+    a.skip_block = p.skip_block;
     // the workspace header (maxima, barrier counter) starts at zero, unless
     // the launch uses none of it: MXFP4 without a norm, or a given amax with
     // the shared residual scale (one pass, no barrier)

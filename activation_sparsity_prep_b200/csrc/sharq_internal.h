@@ -29,12 +29,16 @@ struct PrepareLaunch {
     float* rs_tscale;
     void* mask;
     void* ws;
+    unsigned long long wait_ns = 0;   // limit of each grid-barrier wait (0: the default, ~1 s)
+    int skip_block = -1;              // self-test only: this block never arrives at a barrier
+    bool spec_off = false;            // NVFP4 own scale: always run phase 3 (for measurements)
 };
 
 size_t prepare_ws_bytes(int64_t M);
 cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms);
-// Failure-path self-test (selftest.cu): a grid wait that one block never
-// joins, bounded by limit_ns.
+// Failure-path self-test (selftest.cu): the library's bounded grid barrier
+// with one block that never arrives, and its bounded mbarrier wait on a
+// phase that never completes, each bounded by limit_ns.
 cudaError_t launch_wait_selftest(uint32_t* counter, unsigned long long limit_ns, cudaStream_t s);
 
 struct LinearLaunch {

@@ -270,13 +270,29 @@ SHARQ_API sharq_status sharq_moe_linear_swiglu(const sharq_prepared* x, const in
 SHARQ_API sharq_status sharq_prepare_noalloc(const void* X_bf16, const void* gamma_bf16, float eps,
                                              const sharq_prepared* out, void* stream);
 
-/* Self-test of the failure path (for test suites): launches a small grid
- * wait that one block never joins.  Each waiting block gives up after
- * limit_us microseconds (1000 .. 1000000), records a timeout in the device
- * status word and returns, so the next sharq_last_device_status() reports
- * SHARQ_ERR_TIMEOUT and the context stays usable.  ws: device memory of at
- * least 4 bytes (4-byte aligned), overwritten.  Nothing faults or hangs. */
+/* Self-test of the failure path (for test suites): runs the library's own
+ * bounded waits into their limit -- its grid barrier over a small grid whose
+ * last block never arrives, then its mbarrier wait on a phase that nothing
+ * completes.  Each wait gives up after limit_us microseconds (1000 ..
+ * 1000000), records a timeout in the device status word and returns, so the
+ * next sharq_last_device_status() reports SHARQ_ERR_TIMEOUT and the context
+ * stays usable.  ws: device memory of at least 4 bytes (4-byte aligned),
+ * overwritten.  Nothing faults or hangs. */
 SHARQ_API sharq_status sharq_selftest_wait_timeout(void* ws, int64_t limit_us, void* stream);
+
+/* Self-test of the failure path inside the preparation operator itself
+ * (for test suites): runs sharq_prepare(X, NULL, ...) -- NVFP4, no norm, own
+ * residual scale, so the launch has its two grid barriers -- with block 0
+ * never arriving at them and every barrier wait limited to limit_us
+ * microseconds (1000 .. 1000000).  The other blocks' waits give up, record
+ * a timeout in the device status word and the kernel runs to its end, so
+ * the next sharq_last_device_status() reports SHARQ_ERR_TIMEOUT; the
+ * outputs of this call are unspecified and nothing faults or hangs.
+ * Arguments as sharq_prepare; out->fmt must be SHARQ_NVFP4 and
+ * out->residual_scale SHARQ_RESIDUAL_OWN, out->M >= 1. */
+SHARQ_API sharq_status sharq_selftest_prepare_timeout(const void* X_bf16, const sharq_prepared* out,
+                                                      void* ws, size_t ws_bytes, int64_t limit_us,
+                                                      void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word:
  * SHARQ_OK, SHARQ_ERR_TIMEOUT if a bounded device wait gave up since the

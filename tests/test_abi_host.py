@@ -184,3 +184,18 @@ def test_wait_selftest_rejects_bad_arguments_on_host():
     assert L.sharq_selftest_wait_timeout(0x1002, 10000, None) == 1      # misaligned
     assert L.sharq_selftest_wait_timeout(0x1000, 10, None) == 1         # below 1 ms
     assert L.sharq_selftest_wait_timeout(0x1000, 5_000_000, None) == 1  # above 1 s
+
+
+def test_prepare_timeout_selftest_rejects_bad_arguments_on_host():
+    L = sq.load_sharq_ops()
+    cp = _fake_prepared()
+    ok = L.sharq_selftest_prepare_timeout(ctypes.c_void_p(0x1000), ctypes.byref(cp), ctypes.c_void_p(0x1000),
+                                          1 << 20, 10, None)
+    assert ok == 1                                                          # limit below 1 ms
+    cp.fmt = 1
+    assert L.sharq_selftest_prepare_timeout(ctypes.c_void_p(0x1000), ctypes.byref(cp), ctypes.c_void_p(0x1000),
+                                            1 << 20, 10000, None) == 1      # MXFP4 has no grid barriers here
+    cp.fmt = 0
+    cp.residual_scale = 1
+    assert L.sharq_selftest_prepare_timeout(ctypes.c_void_p(0x1000), ctypes.byref(cp), ctypes.c_void_p(0x1000),
+                                            1 << 20, 10000, None) == 1      # shared scale: one barrier only

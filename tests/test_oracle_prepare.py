@@ -419,3 +419,34 @@ def test_linear_abs_bruteforce_tiny(fmt, residual):
             assert abs(Y[i, j] - gw * (gb * yb + gr * yr)) <= 1e-12 * want
     # both paths contribute (neither half of the sum was dropped)
     assert np.abs(P.rs.codes & 0x77).sum() > 0 and np.abs(P.bb.codes & 0x77).sum() > 0
+
+
+def _pruned_and_kept_residual_max(X, g, n=2, m=4):
+    y = oracle.normalize(X, g, 1e-6)
+    keep = oracle.mask(y, n, m).astype(bool)
+    R = oracle.prepare(X, g, 1e-6, n, m, "nvfp4")
+    D = (oracle.dequant_blocks(R.bb).astype(np.float32) * np.float32(R.bb.tscale))
+    r = (y - D).astype(np.float32)
+    P = np.abs(np.where(keep, np.float32(0), y)).max()
+    Q = np.abs(np.where(keep, r, np.float32(0))).max()
+    return P, Q, R
+
+
+@pytest.mark.parametrize("dist,gk", [("student_t", None), ("student_t", "ones"),
+                                     ("laplace_outlier", None), ("laplace_outlier", "ones")])
+def test_residual_tensor_max_is_pruned_or_kept_max(dist, gk):
+    """The residual of a pruned entry is y itself and that of a kept entry is
+    y - dequant(backbone), so A_r = max(P, Q) with P the largest pruned |y|
+    and Q the largest kept |y - D|.  The GPU prepare takes P in its first
+    pass and guesses A_r = P; these inputs (the parity cases' distributions)
+    cover both outcomes: P wins for Student-t activations, the kept
+    outliers' quantisation error wins for outlier-channel ones."""
+    X = wl.activation(dist, 21, 5, 128, 4096)
+    g = None if gk is None else wl.gamma_ones(4096)
+    P, Q, R = _pruned_and_kept_residual_max(X, g)
+    A_r = np.float32(max(P, Q))
+    assert np.float32(R.rs.tscale) == (np.float32(1) if A_r == 0 else np.float32(A_r / np.float32(2688)))
+    if dist == "student_t":
+        assert P >= Q
+    else:
+        assert Q > P
