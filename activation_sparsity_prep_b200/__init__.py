@@ -22,7 +22,7 @@ from dataclasses import dataclass
 from typing import Optional
 
 __all__ = [
-    "NVFP4", "MXFP4", "SharqError", "load_sharq_ops", "scale_bytes",
+    "NVFP4", "MXFP4", "SharqError", "load_sharq_ops", "scale_bytes", "pair_meta_bytes",
     "prepare_workspace_bytes", "Weight", "Prepared", "quantize_weight",
     "prepare", "prepare_layernorm", "prepare_amax", "prepare_noalloc", "linear",
     "linear_swiglu", "interleave_gate_up", "moe_linear", "moe_linear_swiglu",
@@ -55,7 +55,7 @@ class _Prepared(ctypes.Structure):
                 ("rs_scales", ctypes.c_void_p), ("rs_tscale", ctypes.c_void_p),
                 ("mask", ctypes.c_void_p), ("M", ctypes.c_int), ("K", ctypes.c_int),
                 ("n", ctypes.c_int), ("m", ctypes.c_int), ("fmt", ctypes.c_int),
-                ("residual_scale", ctypes.c_int)]
+                ("residual_scale", ctypes.c_int), ("bb_meta", ctypes.c_void_p)]
 
 
 _lib = None
@@ -85,6 +85,8 @@ def load_sharq_ops(build_if_missing: bool = True) -> ctypes.CDLL:
         L.sharq_scale_bytes.restype = SZ
         L.sharq_prepare_workspace_bytes.argtypes = [I64, I, I]
         L.sharq_prepare_workspace_bytes.restype = SZ
+        L.sharq_pair_meta_bytes.argtypes = [I64, I]
+        L.sharq_pair_meta_bytes.restype = SZ
         L.sharq_quantize_weight.argtypes = [P, ctypes.POINTER(_Weight), P, SZ, P]
         L.sharq_quantize_weight.restype = I
         L.sharq_prepare.argtypes = [P, P, ctypes.c_float, ctypes.POINTER(_Prepared), P, SZ, P]
@@ -200,7 +202,9 @@ def _check_prepared_buffers(p: "Prepared", device=None):
     dev = device if device is not None else p.bb_codes.device
     sb = scale_bytes(p.M, p.K, p.fmt)
     u8 = torch.uint8
-    _check_min("bb_codes", p.bb_codes, p.M * p.K // 2, u8, dev)
+    _check_min("bb_codes", p.bb_codes, p.M * p.K // (4 if p.bb_meta is not None else 2), u8, dev)
+    if p.bb_meta is not None:
+        _check_min("bb_meta", p.bb_meta, pair_meta_bytes(p.M, p.K), u8, dev)
     _check_min("rs_codes", p.rs_codes, p.M * p.K // 2, u8, dev)
     _check_min("bb_scales", p.bb_scales, sb, u8, dev)
     _check_min("rs_scales", p.rs_scales, sb, u8, dev)
@@ -226,6 +230,11 @@ def _check_output(name: str, Y, shape, dtype, device):
 
 def scale_bytes(rows: int, K: int, fmt="nvfp4") -> int:
     return int(load_sharq_ops().sharq_scale_bytes(rows, K, _fmt(fmt)))
+
+
+def pair_meta_bytes(M: int, K: int) -> int:
+    """Bytes of the pair metadata of a compressed (pair-granular 4:8) backbone."""
+    return int(load_sharq_ops().sharq_pair_meta_bytes(M, K))
 
 
 def prepare_workspace_bytes(M: int, K: int, fmt="nvfp4") -> int:
@@ -274,26 +283,33 @@ class Prepared:
     m: int
     fmt: int
     residual_scale: int = 0      # 0 own, 1 shared with the backbone (NVFP4)
+    bb_meta: "object" = None     # pair metadata: the backbone is the compressed pair-granular 4:8 form
 
     def _c(self) -> _Prepared:
         return _Prepared(_ptr(self.bb_codes), _ptr(self.bb_scales), _ptr(self.bb_tscale),
                          _ptr(self.rs_codes), _ptr(self.rs_scales), _ptr(self.rs_tscale),
                          _ptr(self.mask), self.M, self.K, self.n, self.m, self.fmt,
-                         self.residual_scale)
+                         self.residual_scale, _ptr(self.bb_meta))
 
     @staticmethod
     def empty(M: int, K: int, n: int = 2, m: int = 4, fmt="nvfp4", want_mask: bool = False,
-              device="cuda", residual_scale="own") -> "Prepared":
+              device="cuda", residual_scale="own", pairs: bool = False) -> "Prepared":
+        """pairs: the pair-granular 4:8 backbone of the FP4 sparse MMA (MXFP4):
+        bb_codes holds the kept pairs [M, K/4] and bb_meta their indices."""
         import torch
         f = _fmt(fmt)
+        if pairs:
+            _need(f == MXFP4, "the pair-granular backbone is MXFP4")
+            n, m = 4, 8
         sb = scale_bytes(M, K, f)
         u8 = dict(dtype=torch.uint8, device=device)
-        return Prepared(torch.empty((M, K // 2), **u8), torch.empty((sb,), **u8),
+        return Prepared(torch.empty((M, K // 4 if pairs else K // 2), **u8), torch.empty((sb,), **u8),
                         torch.empty((1,), dtype=torch.float32, device=device),
                         torch.empty((M, K // 2), **u8), torch.empty((sb,), **u8),
                         torch.empty((1,), dtype=torch.float32, device=device),
                         torch.empty((M, K // 8), **u8) if want_mask else None,
-                        M, K, n, m, f, _residual(residual_scale))
+                        M, K, n, m, f, _residual(residual_scale),
+                        torch.empty((pair_meta_bytes(M, K),), **u8) if pairs else None)
 
 
 def _workspace(M: int, K: int, fmt: int, ws=None, device="cuda"):
@@ -324,10 +340,13 @@ def quantize_weight(W, fmt="nvfp4", out: Optional[Weight] = None, ws=None, strea
 
 def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4",
             want_mask: bool = False, out: Optional[Prepared] = None, ws=None,
-            stream=None, residual_scale="own") -> Prepared:
+            stream=None, residual_scale="own", pairs: bool = False) -> Prepared:
     """X: bf16 [M, K] device tensor; gamma: bf16 [K] or None (no norm).
     residual_scale: "own" or "shared" (ignored when ``out`` is given: the
-    output's own setting applies)."""
+    output's own setting applies).  pairs: the pair-granular 4:8 backbone
+    (MXFP4; n and m are then 4 and 8), compressed for the sparse MMA."""
+    if pairs:
+        fmt, n, m = "mxfp4", 4, 8
     L = load_sharq_ops()
     _check_input(X, gamma)
     M, K = X.shape
@@ -335,7 +354,7 @@ def prepare(X, gamma=None, eps: float = 1e-6, n: int = 2, m: int = 4, fmt="nvfp4
     if out is not None:
         _check_prepared(out, M, K, f, X.device)
     p = out if out is not None else Prepared.empty(M, K, n, m, f, want_mask, device=X.device,
-                                                   residual_scale=residual_scale)
+                                                   residual_scale=residual_scale, pairs=pairs)
     ws = _workspace(M, K, f, ws, X.device)
     cp = p._c()
     _check("sharq_prepare",

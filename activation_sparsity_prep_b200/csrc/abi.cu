@@ -62,6 +62,11 @@ size_t sharq_scale_bytes(int64_t rows, int K, int fmt) {
     return (size_t)(rpad * (K / block_size(fmt)));
 }
 
+size_t sharq_pair_meta_bytes(int64_t rows, int K) {
+    if (!valid_shape(rows, K)) return 0;
+    return (size_t)((rows + 127) / 128 * 128) * (size_t)(K / 16);
+}
+
 size_t sharq_prepare_workspace_bytes(int64_t M, int K, int fmt) {
     if (!valid_fmt(fmt) || !valid_shape(M, K)) return 0;
     return sharq::prepare_ws_bytes(M);
@@ -108,8 +113,15 @@ static sharq_status prepare_common(const void* X_bf16, const void* gamma_bf16, c
         ((uintptr_t)o.rs_tscale & 3u))
         return SHARQ_ERR_INVALID_ARG;
     if (ws_bytes < sharq::prepare_ws_bytes(o.M)) return SHARQ_ERR_INVALID_ARG;
+    if (o.bb_meta) {
+        // pair-granular 4:8 backbone: MXFP4, RMSNorm or no norm, the norm computed here
+        if (o.fmt != SHARQ_MXFP4 || o.n != 4 || o.m != 8) return SHARQ_ERR_INVALID_ARG;
+        if (!aligned16(o.bb_meta)) return SHARQ_ERR_INVALID_ARG;
+        if (layernorm || amax || skip_block >= 0) return SHARQ_ERR_UNSUPPORTED;
+    }
     sharq::PrepareLaunch p{};
     p.X = X_bf16; p.gamma = gamma_bf16; p.eps = eps; p.M = o.M; p.K = o.K; p.n = o.n; p.m = o.m;
+    p.bb_meta = o.bb_meta;
     p.beta = layernorm ? beta_bf16 : nullptr; p.layernorm = layernorm;
     p.fmt = o.fmt; p.weight = false; p.residual_shared = o.residual_scale == SHARQ_RESIDUAL_SHARED;
     p.bb_codes = o.bb_codes; p.bb_scales = o.bb_scales; p.bb_tscale = o.bb_tscale;
@@ -151,6 +163,7 @@ static sharq_status check_linear_args(const sharq_prepared* x, const sharq_weigh
     if (!aligned16(x->bb_codes) || !aligned16(x->bb_scales) || !aligned16(x->rs_codes) ||
         !aligned16(x->rs_scales) || !aligned16(w->codes) || !aligned16(w->scales) || !aligned16(Y))
         return SHARQ_ERR_INVALID_ARG;
+    if (x->bb_meta && (x->fmt != SHARQ_MXFP4 || !aligned16(x->bb_meta))) return SHARQ_ERR_INVALID_ARG;
     return SHARQ_OK;
 }
 
@@ -161,6 +174,7 @@ sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight* w, void* 
     if (x->M == 0) return SHARQ_OK;
     sharq::LinearLaunch p{};
     p.bb_codes = x->bb_codes; p.bb_scales = x->bb_scales; p.bb_tscale = x->bb_tscale;
+    p.bb_meta = x->bb_meta;
     p.rs_codes = x->rs_codes; p.rs_scales = x->rs_scales; p.rs_tscale = x->rs_tscale;
     p.w_codes = w->codes; p.w_scales = w->scales; p.w_tscale = w->tensor_scale;
     p.M = x->M; p.N = w->N; p.K = x->K; p.fmt = x->fmt; p.Y = Y; p.y_fp32 = y_is_fp32 ? 1 : 0;
@@ -174,6 +188,7 @@ sharq_status sharq_linear_swiglu(const sharq_prepared* x, const sharq_weight* w,
     sharq_status st = check_linear_args(x, w, H);
     if (st != SHARQ_OK) return st;
     if (!h_amax || ((uintptr_t)h_amax & 3u)) return SHARQ_ERR_INVALID_ARG;
+    if (x->bb_meta) return SHARQ_ERR_UNSUPPORTED;
     if (x->M == 0)
         return cuda_status(cudaMemsetAsync(h_amax, 0, sizeof(float), static_cast<cudaStream_t>(stream)));
     sharq::LinearLaunch p{};
@@ -198,6 +213,7 @@ static sharq_status moe_common(const sharq_prepared* x, const int32_t* row_index
                                void* stream) {
     if (!x || !w) return SHARQ_ERR_INVALID_ARG;
     if (!expert_offsets || E <= 0 || T < 0 || (!row_index && T != x->M)) return SHARQ_ERR_INVALID_ARG;
+    if (x->bb_meta) return SHARQ_ERR_UNSUPPORTED;
     if (E > 256) return SHARQ_ERR_UNSUPPORTED;
     if (T > 0 && (!Y || !ws)) return SHARQ_ERR_INVALID_ARG;
     if (!valid_fmt(x->fmt) || x->fmt != w->fmt || !valid_shape(x->M, x->K) || x->K != w->K)

@@ -275,6 +275,20 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
                     "r"(sfa_tmem), "r"(sfb_tmem) : "memory");
 }
 
+// Sparse A (pair-granular 4:8: A holds the kept pairs, 64 stored = 128
+// logical elements of K per instruction, their pair indices at tensor-memory
+// address meta_tmem), dense B; E2M1 operands with a block scale per 16
+// stored = 32 logical elements, E4M3 or E8M0 by the instruction descriptor.
+__device__ __forceinline__ void tc_mma_sp_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t meta_tmem, uint32_t idesc, uint32_t sfa_tmem,
+                                               uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16"
+                 " [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}"
+                 :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
+                    "r"(sfa_tmem), "r"(sfb_tmem), "r"(meta_tmem) : "memory");
+}
+
 // Same with E8M0 scales per 32 (MXFP4).
 __device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
@@ -319,6 +333,10 @@ __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint4 (&
                  :: "r"(taddr), "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w),
                     "r"(v[1].x), "r"(v[1].y), "r"(v[1].z), "r"(v[1].w) : "memory");
 }
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+                 :: "r"(taddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint4 (&v)[4]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, "
                  "%9, %10, %11, %12, %13, %14, %15, %16};"
@@ -355,5 +373,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return d;
 }
 
+
+// The same for rows of 64 bytes with the 64-byte swizzle: 8-row groups 512
+// bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);          // start address, bits 0-13
+    d |= (uint64_t)(16u >> 4) << 16;                  // leading byte offset (unused with swizzle)
+    d |= (uint64_t)(512u >> 4) << 32;                 // stride byte offset: 8 rows x 64 B
+    d |= (uint64_t)1 << 46;                           // descriptor version (sm_100)
+    d |= (uint64_t)4 << 61;                           // layout: 64-byte swizzle
+    return d;
+}
 
 }  // namespace sharq

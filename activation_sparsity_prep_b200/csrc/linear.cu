@@ -58,6 +58,28 @@ struct Cfg {
                                        ((uint32_t)FMT << 23) | ((uint32_t)(BM >> 4) << 24);
 };
 
+// Stage of the sparse-backbone form (MXFP4, pair-granular 4:8 backbone):
+// the backbone tile holds only the kept pairs, 64 bytes per row (64-byte
+// swizzle), followed by the residual and weight tiles, the three scale
+// groups and the 128-row x 16-byte pair-metadata atom of the k-step.
+struct SpStage {
+    static constexpr uint32_t kBc = 0;                         // compressed backbone, 8 KiB
+    static constexpr uint32_t kRs = BM * (BK / 4);             // residual tile, 16 KiB
+    static constexpr uint32_t kW = kRs + kTileBytes;            // weight tile, 16 KiB
+    static constexpr uint32_t kSf = kW + kTileBytes;            // 3 x 1 KiB of E8M0 scale atoms
+    static constexpr uint32_t kSfBytes = Cfg<1>::kSfBytes;
+    static constexpr uint32_t kMeta = kSf + 3 * kSfBytes;       // 2 KiB of pair indices
+    static constexpr uint32_t kMetaBytes = BM * 16;
+    static constexpr uint32_t kBytes = kMeta + kMetaBytes;
+    static constexpr uint32_t kStride = (kBytes + 1023) / 1024 * 1024;
+    // sparse MMA: E2M1 A and B, E8M0 scales per 32 logical elements
+    // (block16 of stored elements), sparse flag, N and M as the dense form
+    static constexpr uint32_t kIdesc = (1u << 2) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                       (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+};
+static_assert(SpStage::kStride % 1024 == 0 && SpStage::kRs % 1024 == 0 && SpStage::kW % 1024 == 0,
+              "swizzled tiles start on 1 KiB boundaries");
+
 struct alignas(8) Barriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];      // MMAs done (tcgen05.commit) + scale warps done reading
@@ -223,16 +245,22 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
 // thread waits only until the epilogue has copied the previous tile's two
 // accumulators out of tensor memory, so the epilogue's global stores overlap
 // the next tile's MMAs.
-template <int FMT, bool ONE, bool SW>
+// SPB: the backbone is the compressed pair-granular 4:8 form (MXFP4 only):
+// per k-step two sparse MMAs (128 logical K each, pair indices in tensor
+// memory) on the backbone and four dense MMAs on the residual, all into one
+// accumulator and all on the same weight tile.
+template <int FMT, bool ONE, bool SW, bool SPB>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_r,
               const __grid_constant__ CUtensorMap tm_w, const uint8_t* __restrict__ sf_b,
-              const uint8_t* __restrict__ sf_r, const uint8_t* __restrict__ sf_w, int K,
-              EpiArgs ep, Sched sc) {
+              const uint8_t* __restrict__ sf_r, const uint8_t* __restrict__ sf_w,
+              const uint8_t* __restrict__ meta, int K, EpiArgs ep, Sched sc) {
     using C = Cfg<FMT>;
+    static_assert(!SPB || (FMT == 1 && ONE && !SW), "sparse backbone: MXFP4, one accumulator");
+    constexpr uint32_t kStride = SPB ? SpStage::kStride : C::kStageStride;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Barriers* bars = reinterpret_cast<Barriers*>(smem + kStages * C::kStageStride);
+    Barriers* bars = reinterpret_cast<Barriers*>(smem + kStages * kStride);
     // 128-byte aligned: the staging buffers take 16-byte vector stores
     SchedSmem* ssm = reinterpret_cast<SchedSmem*>(
         (reinterpret_cast<uintptr_t>(bars) + sizeof(Barriers) + 127) & ~uintptr_t(127));
@@ -267,7 +295,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     // that the block-scaled MMA reads.  Copying them with tcgen05.cp would
     // put 3 * kAtoms copies per stage into the MMA issue stream, where they
     // do not overlap the MMAs.
-    constexpr uint32_t kSfColsPerStage = 3 * 4 * C::kAtoms;
+    constexpr uint32_t kScaleCols = 3 * 4 * C::kAtoms;
+    constexpr uint32_t kSfColsPerStage = kScaleCols + (SPB ? 4 : 0);   // + the pair indices
     static_assert(2 * BN + kStages * kSfColsPerStage <= kTmemCols, "tensor memory budget");
 
     if (warp == 0) {
@@ -283,15 +312,30 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     if (it >= kStages && !mbar_wait(&bars->empty[s], ((it / kStages) - 1) & 1)) { ok = false; break; }
-                    uint8_t* st = smem + s * C::kStageStride;
-                    mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
-                    tma_load_2d(st, &tm_b, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
-                    tma_load_2d(st + kTileBytes, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
-                    tma_load_2d(st + 2 * kTileBytes, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
+                    uint8_t* st = smem + s * kStride;
                     const int64_t sfo = (int64_t)kb * C::kAtoms * 512;
-                    bulk_load(st + 3 * kTileBytes, gb + sfo, C::kSfBytes, &bars->full[s]);
-                    bulk_load(st + 3 * kTileBytes + C::kSfBytes, gr + sfo, C::kSfBytes, &bars->full[s]);
-                    bulk_load(st + 3 * kTileBytes + 2 * C::kSfBytes, gw + sfo, C::kSfBytes, &bars->full[s]);
+                    if constexpr (SPB) {
+                        using P = SpStage;
+                        mbar_arrive_expect_tx(&bars->full[s], P::kBytes);
+                        tma_load_2d(st + P::kBc, &tm_b, &bars->full[s], kb * (BK / 4), (int)ti.a_row);
+                        tma_load_2d(st + P::kRs, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                        tma_load_2d(st + P::kW, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
+                        bulk_load(st + P::kSf, gb + sfo, P::kSfBytes, &bars->full[s]);
+                        bulk_load(st + P::kSf + P::kSfBytes, gr + sfo, P::kSfBytes, &bars->full[s]);
+                        bulk_load(st + P::kSf + 2 * P::kSfBytes, gw + sfo, P::kSfBytes, &bars->full[s]);
+                        // metadata atom (k-step kb, row block a_row / 128)
+                        const int64_t mpad = (sc.M + 127) / 128 * 128;
+                        bulk_load(st + P::kMeta, meta + ((int64_t)kb * (mpad >> 7) + (ti.a_row >> 7)) * 2048,
+                                  P::kMetaBytes, &bars->full[s]);
+                    } else {
+                        mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
+                        tma_load_2d(st, &tm_b, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                        tma_load_2d(st + kTileBytes, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                        tma_load_2d(st + 2 * kTileBytes, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
+                        bulk_load(st + 3 * kTileBytes, gb + sfo, C::kSfBytes, &bars->full[s]);
+                        bulk_load(st + 3 * kTileBytes + C::kSfBytes, gr + sfo, C::kSfBytes, &bars->full[s]);
+                        bulk_load(st + 3 * kTileBytes + 2 * C::kSfBytes, gw + sfo, C::kSfBytes, &bars->full[s]);
+                    }
                 }
             }
         }
@@ -312,12 +356,36 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                     if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
                     if (!mbar_wait(&bars->sf_full[s], (it / kStages) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    uint8_t* st = smem + s * C::kStageStride;
-                    const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + kTileBytes);
-                    const uint32_t a_w = smem_u32(st + 2 * kTileBytes);
+                    uint8_t* st = smem + s * kStride;
                     const uint32_t t_sfa_b = tmem + 2 * BN + s * kSfColsPerStage;
                     const uint32_t t_sfa_r = t_sfa_b + 4 * C::kAtoms;
                     const uint32_t t_sfb = t_sfa_r + 4 * C::kAtoms;
+                    if constexpr (SPB) {
+                        using P = SpStage;
+                        const uint32_t a_bc = smem_u32(st + P::kBc), a_r = smem_u32(st + P::kRs);
+                        const uint32_t a_w = smem_u32(st + P::kW);
+                        const uint32_t t_meta = t_sfa_b + kScaleCols;
+                        // backbone: two sparse MMAs of 128 logical K (32 stored
+                        // bytes of A, 64 bytes of B per row; scale atom h holds
+                        // their four scales per row; two metadata columns each)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tc_mma_sp_nvf4(d_b, sdesc_sw64(a_bc + 32 * h), sdesc_sw128(a_w + 64 * h),
+                                           t_meta + 2 * h, P::kIdesc, t_sfa_b + 4 * h, t_sfb + 4 * h,
+                                           (kb | h) ? 1u : 0u);
+                        // residual: four dense MMAs of 64 K on the same weight tile
+#pragma unroll
+                        for (int j = 0; j < BK / 64; ++j) {
+                            const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
+                            mma<FMT>(d_r, sdesc_sw128(a_r + 32 * j), sdesc_sw128(a_w + 32 * j),
+                                     t_sfa_r + 4 * (j / C::kStepsPerAtom), t_sfb + 4 * (j / C::kStepsPerAtom),
+                                     1u, sf_id);
+                        }
+                        tc_commit(&bars->empty[s]);
+                        continue;
+                    }
+                    const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + kTileBytes);
+                    const uint32_t a_w = smem_u32(st + 2 * kTileBytes);
 #pragma unroll
                     for (int j = 0; j < BK / 64; ++j) {
                         const int at = j / C::kStepsPerAtom;
@@ -345,8 +413,14 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t s = it % kStages;
                 if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
-                const uint8_t* sf = smem + s * C::kStageStride + 3 * kTileBytes;
+                const uint8_t* sf = smem + s * kStride + (SPB ? SpStage::kSf : 3 * kTileBytes);
                 const uint32_t tcol = tmem + 2 * BN + s * kSfColsPerStage + lane_off;
+                if constexpr (SPB) {
+                    // pair indices: tensor-memory lane r holds row r's 16 bytes
+                    // of the stage in K order (four columns)
+                    const uint8_t* mt = smem + s * kStride + SpStage::kMeta;
+                    tmem_st_32x32b_x4(tcol + kScaleCols, ld_shared_v4(mt + 16 * ((warp & 3) * 32 + lane)));
+                }
                 // one store per operand: its kAtoms atoms are 4 * kAtoms
                 // consecutive columns
 #pragma unroll
@@ -825,43 +899,48 @@ cudaError_t set_smem_once(std::atomic<bool> (&done)[64], Fn kernel, size_t bytes
     return e;
 }
 
-// 2-D uint8 map over a [rows, row_bytes] code matrix, box 128 bytes x box_rows,
-// 128-byte swizzle; rows past the end read as zero.
-bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+// 2-D uint8 map over a [rows, row_bytes] code matrix, box box_bytes x
+// box_rows with the swizzle of that row length (128 bytes: 128-byte
+// swizzle; 64 bytes: 64-byte swizzle); rows past the end read as zero.
+bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows,
+                   int box_bytes = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE,
+              box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT>
+template <int FMT, bool SPB = false>
 size_t linear_smem_bytes() {
-    return kStages * Cfg<FMT>::kStageStride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
+    const size_t stride = SPB ? SpStage::kStride : Cfg<FMT>::kStageStride;
+    return kStages * stride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
 }
 
-template <int FMT, bool ONE, bool SW>
+template <int FMT, bool ONE, bool SW, bool SPB = false>
 cudaError_t ensure_smem_attr() {
     static std::atomic<bool> done[64];
-    return set_smem_once(done, linear_kernel<FMT, ONE, SW>, linear_smem_bytes<FMT>());
+    return set_smem_once(done, linear_kernel<FMT, ONE, SW, SPB>, linear_smem_bytes<FMT, SPB>());
 }
 
 // A_rows: rows of the activation operands (gathered and padded for the
 // grouped form); W_rows: rows of the (stacked) weight.
-template <int FMT, bool ONE, bool SW>
+template <int FMT, bool ONE, bool SW, bool SPB = false>
 cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const void* rs_codes,
                         const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
                         const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
     CUtensorMap tb, tr, tw;
-    if (!make_code_map(&tb, bb_codes, A_rows, p.K / 2, BM) ||
+    // the compressed backbone has K/4 bytes a row: 64 bytes a k-step
+    if (!make_code_map(&tb, bb_codes, A_rows, SPB ? p.K / 4 : p.K / 2, BM, SPB ? 64 : 128) ||
         !make_code_map(&tr, rs_codes, A_rows, p.K / 2, BM) ||
         !make_code_map(&tw, p.w_codes, W_rows, p.K / 2, BN))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr<FMT, ONE, SW>();
+    cudaError_t e = ensure_smem_attr<FMT, ONE, SW, SPB>();
     if (e != cudaSuccess) return e;
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32,
                reinterpret_cast<uint32_t*>(p.amax)};
@@ -870,9 +949,9 @@ cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const voi
         if (e != cudaSuccess) return e;
     }
     const int grid = std::max(1, std::min(max_tiles, std::max(1, sms)));
-    linear_kernel<FMT, ONE, SW><<<grid, kThreads, linear_smem_bytes<FMT>(), s>>>(
+    linear_kernel<FMT, ONE, SW, SPB><<<grid, kThreads, linear_smem_bytes<FMT, SPB>(), s>>>(
         tb, tr, tw, static_cast<const uint8_t*>(bb_scales), static_cast<const uint8_t*>(rs_scales),
-        static_cast<const uint8_t*>(p.w_scales), p.K, ep, sc);
+        static_cast<const uint8_t*>(p.w_scales), static_cast<const uint8_t*>(p.bb_meta), p.K, ep, sc);
     return cudaGetLastError();
 }
 
@@ -935,6 +1014,20 @@ cudaError_t launch_decode_nt(const LinearLaunch& p, cudaStream_t s, int sms) {
 
 template <int FMT>
 cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
+    if (p.bb_meta) {
+        // compressed pair-granular backbone: the row-tiled kernel with the
+        // sparse MMA (the swapped decode form would need the backbone as B)
+        if (FMT != 1 || !p.one_acc || p.swiglu) return cudaErrorNotSupported;
+        Sched sc{};
+        sc.mt_count = (int)((p.M + BM - 1) / BM);
+        sc.nt_count = p.N / BN;
+        sc.M = p.M;
+        sc.nsf = p.K / Cfg<FMT>::BS;
+        sc.grouped = 0;
+        sc.N = p.N;
+        return launch_gemm_t<1, true, false, true>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p,
+                                                   p.N, sc, sc.mt_count * sc.nt_count, s, sms);
+    }
     // few rows: the swapped (weight-streaming) form; the SwiGLU epilogue
     // exists in the row-tiled form only
     if (!p.swiglu) {

@@ -55,6 +55,7 @@ extern "C" SHARQ_API sharq_status sharq_prepare_noalloc(const void* X_bf16, cons
                                                         void* stream) {
     if (!out) return SHARQ_ERR_INVALID_ARG;
     const sharq_prepared& o = *out;
+    if (o.bb_meta) return SHARQ_ERR_UNSUPPORTED;   // the compressed pair backbone is not offered here
     if (o.M < 0 || o.M > SHARQ_NOALLOC_MAX_ROWS) return SHARQ_ERR_INVALID_ARG;   // beyond the fixed scratch
     if (!(o.fmt == SHARQ_NVFP4 || o.fmt == SHARQ_MXFP4) || o.K <= 0 || o.K % 256 != 0)
         return SHARQ_ERR_INVALID_ARG;

@@ -65,6 +65,7 @@ struct PrepArgs {
     uint32_t* ws;            // [0] amax_b bits, [1] amax_r bits, [2] barrier, [5] phase-2 guess
                              // failed, [6] max pruned |y| bits; from word 16: rinv[M], mu[M]
     const float* amax_in;    // GIVEN: A_b = max |X| from the producer
+    uint8_t* bb_meta;        // PAIRS: pair metadata atoms (bb_codes then holds the kept pairs)
     int staged;              // gamma (and beta) are in shared memory as fp32
     int spec;                // NVFP4 own residual scale: quantise the residual in phase 2 against
                              // the largest pruned |y| (see phase 2)
@@ -376,6 +377,31 @@ __device__ __forceinline__ uint32_t keep24_nibbles8(const float* y) {
     return lop3t<0xE4>(ev, od, 0x0F0F0F0Fu);      // (ev & 0x0F..) | (od & 0xF0..)
 }
 
+// The pair-granular 4:8 mask of 8 elements: the two of the four aligned
+// pairs with the largest pair magnitude max(|y_2i|, |y_2i+1|), ties to the
+// lower pair index (the same majority functions as keep24_nibbles8, on the
+// pair magnitudes).  Returns the code AND mask (0xFF in byte i, the codes
+// of pair i, when it is kept) and in *nib the metadata nibble: the lower
+// kept pair's index in bits 1:0, the higher one's in bits 3:2.
+__device__ __forceinline__ uint32_t keep_pairs_bytes8(const float* y, uint32_t* nib) {
+    const float a0 = fmaxf(fabsf(y[0]), fabsf(y[1])), a1 = fmaxf(fabsf(y[2]), fabsf(y[3]));
+    const float a2 = fmaxf(fabsf(y[4]), fabsf(y[5])), a3 = fmaxf(fabsf(y[6]), fabsf(y[7]));
+    const uint32_t d01 = __float_as_uint(__fsub_rn(a0, a1)), d02 = __float_as_uint(__fsub_rn(a0, a2));
+    const uint32_t d03 = __float_as_uint(__fsub_rn(a0, a3)), d12 = __float_as_uint(__fsub_rn(a1, a2));
+    const uint32_t d13 = __float_as_uint(__fsub_rn(a1, a3)), d23 = __float_as_uint(__fsub_rn(a2, a3));
+    const uint32_t k0 = lop3t<0x17>(d01, d02, d03), k1 = lop3t<0x71>(d01, d12, d13);
+    const uint32_t k2 = lop3t<0xD4>(d02, d12, d23), k3 = lop3t<0xE8>(d03, d13, d23);
+    const uint32_t m = prmt(prmt(k0, k1, 0x00FBu), prmt(k2, k3, 0xFB00u), 0x7610u);
+    // the four keep bits (bit i = pair i), then the nibble of the two kept
+    // indices: 0b0011 -> 0x4, 0b0101 -> 0x8, 0b0110 -> 0x9, 0b1001 -> 0xC,
+    // 0b1010 -> 0xD, 0b1100 -> 0xE
+    const uint32_t k4 = ((m & 0x01010101u) * 0x01020408u) >> 24;
+    constexpr unsigned long long kLut = (0x4ull << 12) | (0x8ull << 20) | (0x9ull << 24) |
+                                        (0xCull << 36) | (0xDull << 40) | (0xEull << 48);
+    *nib = (uint32_t)(kLut >> (4 * k4)) & 0xFu;
+    return m;
+}
+
 // Keep bits (bit t = element t) of a code AND mask (0xF in nibble t).
 __device__ __forceinline__ uint32_t nibbles_to_bits8(uint32_t m) {
     uint32_t b = 0;
@@ -469,7 +495,8 @@ struct LaneBlock {
 // phase 2 with the backbone's reciprocal table and phase 3 does not exist.
 // GIVEN: no norm, A_b read from a.amax_in, no phase 1.
 // ------------------------------------------------------------------------
-template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS, bool LN, bool GIVEN>
+template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS, bool LN, bool GIVEN,
+          bool PAIRS>
 __global__ void __launch_bounds__(kThreads, 2)
 prepare_kernel(PrepArgs a) {
     __shared__ float s_inv[128];
@@ -480,6 +507,7 @@ prepare_kernel(PrepArgs a) {
     using LB = LaneBlock<FMT, HAS_GAMMA, LN>;
     static_assert(!LN || HAS_GAMMA, "LayerNorm takes gamma");
     static_assert(!GIVEN || (FMT == 0 && !HAS_GAMMA && !WEIGHT), "a given amax: NVFP4, no norm");
+    static_assert(!PAIRS || (FMT == 1 && !WEIGHT && !LN), "pair backbone: MXFP4 activations");
     const bool has_beta = LN && a.beta != nullptr;
     constexpr int E = LB::E;
 
@@ -666,6 +694,17 @@ prepare_kernel(PrepArgs a) {
             *reinterpret_cast<uint32_t*>(a.bb_scales + sf_off(row, s4 * 4, nsf)) = 0u;
             if (!WEIGHT) *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, s4 * 4, nsf)) = 0u;
         }
+        if (PAIRS) {
+            // padding rows of the metadata atoms: pairs 0 and 1 (of zero codes)
+            const int kblk = K / 256;
+            const int64_t nmeta = (Mpad - M) * kblk;
+            for (int64_t i = gwarp * 32 + lane; i < nmeta; i += nwarps * 32) {
+                const int64_t row = M + i / kblk;
+                const int kb = (int)(i % kblk);
+                *reinterpret_cast<uint4*>(a.bb_meta + ((int64_t)kb * (Mpad >> 7) + (row >> 7)) * 2048 +
+                                          (row & 127) * 16) = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+            }
+        }
     }
 
     const int nb_row = K / E;
@@ -721,9 +760,11 @@ prepare_kernel(PrepArgs a) {
             }
             // the mask as one code AND mask (0xF per kept element) per 8 elements
             uint32_t kmask[E / 8];
+            uint32_t pnib[E / 8];          // PAIRS: metadata nibble of each group of 8
 #pragma unroll
             for (int v = 0; v < E / 8; ++v) {
                 if (WEIGHT)     kmask[v] = 0xFFFFFFFFu;
+                else if (PAIRS) kmask[v] = keep_pairs_bytes8(y + 8 * v, &pnib[v]);
                 else if (NM24)  kmask[v] = keep24_nibbles8(y + 8 * v);
                 else            kmask[v] = nibble_mask8(keep_bits<8, MG, NM24>(y + 8 * v, a.n));
             }
@@ -736,9 +777,23 @@ prepare_kernel(PrepArgs a) {
                 for (int p = 0; p < 4; ++p) q[p] = mul2_rn(y2[4 * v + p], inv2);
                 codes[v] = cvt_e2m1x8_f2(q) & kmask[v];   // pruned: code 0 (+0)
             }
-            uint8_t* cp = a.bb_codes + row * (K / 2) + (int64_t)cb * (E / 2);
-            if (E == 16) *reinterpret_cast<uint2*>(cp) = make_uint2(codes[0], codes[1]);
-            else         *reinterpret_cast<uint4*>(cp) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            if constexpr (PAIRS) {
+                // the kept pairs' code bytes in order (8 bytes for the 32
+                // elements), and the four metadata nibbles into the atom
+                uint32_t kept[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    kept[v] = prmt(codes[v], 0u, (pnib[v] & 3u) | ((pnib[v] >> 2) << 4) | 0x4400u);
+                *reinterpret_cast<uint2*>(a.bb_codes + row * (K / 4) + (int64_t)cb * 8) =
+                    make_uint2(kept[0] | (kept[1] << 16), kept[2] | (kept[3] << 16));
+                const uint32_t nib16 = pnib[0] | (pnib[1] << 4) | (pnib[2] << 8) | (pnib[3] << 12);
+                *reinterpret_cast<uint16_t*>(a.bb_meta + ((int64_t)(cb >> 3) * (Mpad >> 7) + (row >> 7)) * 2048 +
+                                             (row & 127) * 16 + 2 * (cb & 7)) = (uint16_t)nib16;
+            } else {
+                uint8_t* cp = a.bb_codes + row * (K / 2) + (int64_t)cb * (E / 2);
+                if (E == 16) *reinterpret_cast<uint2*>(cp) = make_uint2(codes[0], codes[1]);
+                else         *reinterpret_cast<uint4*>(cp) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            }
             a.bb_scales[cur.sfo] = (uint8_t)ecode;
             if (!WEIGHT && a.mask) {
                 uint8_t* mp = a.mask + row * (K / 8) + (int64_t)cb * (E / 8);
@@ -890,9 +945,9 @@ prepare_kernel(PrepArgs a) {
 }
 
 template <int FMT, bool HAS_GAMMA, int MG, bool WEIGHT, bool NM24, bool RS = false, bool LN = false,
-          bool GIVEN = false>
+          bool GIVEN = false, bool PAIRS = false>
 cudaError_t launch_one(const PrepArgs& a, cudaStream_t s, int max_blocks) {
-    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN, GIVEN>;
+    auto kfn = prepare_kernel<FMT, HAS_GAMMA, MG, WEIGHT, NM24, RS, LN, GIVEN, PAIRS>;
     const size_t smem = a.staged ? (size_t)a.K * 4 * (LN && a.beta ? 2 : 1) : 0;
     // Resident blocks per SM at this shared-memory size (the cooperative
     // grid must not exceed it); the same for every device of one
@@ -976,6 +1031,7 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     a.mask = static_cast<uint8_t*>(p.mask);
     a.ws = static_cast<uint32_t*>(p.ws);
     a.amax_in = p.amax;
+    a.bb_meta = static_cast<uint8_t*>(p.bb_meta);
     const bool g = p.gamma != nullptr;
     const size_t vec_bytes = (size_t)p.K * 4 * (p.layernorm && p.beta ? 2 : 1);
     a.staged = g && vec_bytes <= (size_t)kMaxStagedBytes;
@@ -993,6 +1049,10 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms) {
     if (p.weight) {
         return p.fmt == 0 ? launch_one<0, false, 8, true, false>(a, s, sms)
                           : launch_one<1, false, 8, true, false>(a, s, sms);
+    }
+    if (p.bb_meta) {              // pair-granular 4:8 backbone, MXFP4
+        return g ? launch_one<1, true, 8, false, false, false, false, false, true>(a, s, sms)
+                 : launch_one<1, false, 8, false, false, false, false, false, true>(a, s, sms);
     }
     if (p.layernorm) {
         if (p.fmt == 1) return launch_m<1, true, false, false, true>(a, p.m, s, sms);

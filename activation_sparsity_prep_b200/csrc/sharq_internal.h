@@ -29,6 +29,7 @@ struct PrepareLaunch {
     float* rs_tscale;
     void* mask;
     void* ws;
+    void* bb_meta = nullptr;          // pair-granular 4:8 backbone: bb_codes compressed, metadata here
     unsigned long long wait_ns = 0;   // limit of each grid-barrier wait (0: the default, ~1 s)
     int skip_block = -1;              // self-test only: this block never arrives at a barrier
     bool spec_off = false;            // NVFP4 own scale: always run phase 3 (for measurements)
@@ -42,9 +43,10 @@ cudaError_t launch_prepare(const PrepareLaunch& p, cudaStream_t s, int sms);
 cudaError_t launch_wait_selftest(uint32_t* counter, unsigned long long limit_ns, cudaStream_t s);
 
 struct LinearLaunch {
-    const void* bb_codes;
+    const void* bb_codes;     // compressed [M, K/4] when bb_meta is set
     const void* bb_scales;
     const float* bb_tscale;
+    const void* bb_meta;      // pair metadata atoms of a compressed backbone, or null
     const void* rs_codes;
     const void* rs_scales;
     const float* rs_tscale;

@@ -108,7 +108,28 @@ typedef struct {
     int    M, K, n, m;
     int    fmt;          /* sharq_format */
     int    residual_scale;   /* sharq_residual_scale (0 = OWN)              */
+    void*  bb_meta;      /* NULL: the backbone is zero-filled codes [M, K/2]
+                            under the element-wise n:m mask.  Non-NULL: the
+                            pair-granular 4:8 backbone of the FP4 sparse
+                            MMA (MXFP4 only, n = 4, m = 8): in every aligned
+                            group of 8 elements the two pairs of largest
+                            pair magnitude max(|y_2i|, |y_2i+1|) are kept
+                            (ties: lower pair index); bb_codes then holds
+                            the kept pairs' code bytes in order, [M, K/4],
+                            and bb_meta their pair indices,
+                            sharq_pair_meta_bytes(M, K) bytes (layout
+                            below).                                         */
 } sharq_prepared;
+
+/* Pair metadata of a compressed backbone (bb_meta): per group of 8
+ * elements a nibble with the lower kept pair's index in bits 1:0 and the
+ * higher one's in bits 3:2; group 2j of a row's 256-element K block in the
+ * low nibble of byte j.  Stored in MMA-ready atoms of 128 rows x 256
+ * elements (16 bytes per row, row r at byte 16 * (r % 128)), atom
+ * (k-block kb, row block rb) at byte (kb * rows_pad / 128 + rb) * 2048,
+ * rows padded to a multiple of 128 (padding rows hold 0x44: pairs 0 and 1
+ * of zero codes). */
+SHARQ_API size_t sharq_pair_meta_bytes(int64_t rows, int K);
 
 /* Human-readable name of a status code (static string). */
 SHARQ_API const char* sharq_status_string(int status);

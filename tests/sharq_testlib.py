@@ -42,3 +42,26 @@ def to_np(t):
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).cpu().numpy().view(np.uint16)
     return t.cpu().numpy()
+
+
+def meta_atom_index(rows, K):
+    """Byte offsets of canonical pair metadata (r, j) ([rows, K/16], group 2j
+    of a row in the low nibble of byte j) inside the atom buffer: atom
+    (k-block j // 16, row block r // 128) at ((j // 16) * rows_pad / 128 +
+    r // 128) * 2048, row r % 128 at 16 bytes a row (layout of include/sharq.h)."""
+    rp = (rows + 127) // 128 * 128
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    j = np.arange(K // 16, dtype=np.int64)[None, :]
+    return ((j // 16) * (rp // 128) + r // 128) * 2048 + (r % 128) * 16 + j % 16
+
+
+def meta_atoms_to_canonical(buf, rows, K):
+    return np.asarray(buf).reshape(-1)[meta_atom_index(rows, K)]
+
+
+def canonical_to_meta_atoms(meta, K):
+    rows = meta.shape[0]
+    rp = (rows + 127) // 128 * 128
+    out = np.full(rp * (K // 16), 0x44, dtype=np.uint8)
+    out[meta_atom_index(rows, K)] = meta
+    return out
