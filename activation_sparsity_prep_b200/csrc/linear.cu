@@ -81,7 +81,8 @@ static_assert(SpStage::kStride % 1024 == 0 && SpStage::kRs % 1024 == 0 && SpStag
               "swizzled tiles start on 1 KiB boundaries");
 
 struct alignas(8) Barriers {
-    uint64_t full[kStages];
+    uint64_t full[kStages];       // the stage's operand tiles have landed
+    uint64_t sfl[kStages];        // the stage's scale atoms (and pair indices) have landed
     uint64_t empty[kStages];      // MMAs done (tcgen05.commit) + scale warps done reading
     uint64_t sf_full[kStages];    // scale factors of the stage are in tensor memory
     uint64_t acc_full[2];   // MMAs of a tile done (tcgen05.commit), per accumulator buffer
@@ -273,6 +274,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->sfl[s], 1);
             mbar_init(&bars->empty[s], 1 + 4);
             mbar_init(&bars->sf_full[s], 4);
         }
@@ -314,27 +316,32 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                     if (it >= kStages && !mbar_wait(&bars->empty[s], ((it / kStages) - 1) & 1)) { ok = false; break; }
                     uint8_t* st = smem + s * kStride;
                     const int64_t sfo = (int64_t)kb * C::kAtoms * 512;
+                    // The scale bytes come first, on their own barrier, so the
+                    // scale warps stage them into tensor memory while the
+                    // operand tiles are still arriving.
                     if constexpr (SPB) {
                         using P = SpStage;
-                        mbar_arrive_expect_tx(&bars->full[s], P::kBytes);
-                        tma_load_2d(st + P::kBc, &tm_b, &bars->full[s], kb * (BK / 4), (int)ti.a_row);
-                        tma_load_2d(st + P::kRs, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
-                        tma_load_2d(st + P::kW, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
-                        bulk_load(st + P::kSf, gb + sfo, P::kSfBytes, &bars->full[s]);
-                        bulk_load(st + P::kSf + P::kSfBytes, gr + sfo, P::kSfBytes, &bars->full[s]);
-                        bulk_load(st + P::kSf + 2 * P::kSfBytes, gw + sfo, P::kSfBytes, &bars->full[s]);
+                        mbar_arrive_expect_tx(&bars->sfl[s], P::kBytes - P::kSf);
+                        bulk_load(st + P::kSf, gb + sfo, P::kSfBytes, &bars->sfl[s]);
+                        bulk_load(st + P::kSf + P::kSfBytes, gr + sfo, P::kSfBytes, &bars->sfl[s]);
+                        bulk_load(st + P::kSf + 2 * P::kSfBytes, gw + sfo, P::kSfBytes, &bars->sfl[s]);
                         // metadata atom (k-step kb, row block a_row / 128)
                         const int64_t mpad = (sc.M + 127) / 128 * 128;
                         bulk_load(st + P::kMeta, meta + ((int64_t)kb * (mpad >> 7) + (ti.a_row >> 7)) * 2048,
-                                  P::kMetaBytes, &bars->full[s]);
+                                  P::kMetaBytes, &bars->sfl[s]);
+                        mbar_arrive_expect_tx(&bars->full[s], P::kSf);
+                        tma_load_2d(st + P::kBc, &tm_b, &bars->full[s], kb * (BK / 4), (int)ti.a_row);
+                        tma_load_2d(st + P::kRs, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                        tma_load_2d(st + P::kW, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
                     } else {
-                        mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
+                        mbar_arrive_expect_tx(&bars->sfl[s], 3 * C::kSfBytes);
+                        bulk_load(st + 3 * kTileBytes, gb + sfo, C::kSfBytes, &bars->sfl[s]);
+                        bulk_load(st + 3 * kTileBytes + C::kSfBytes, gr + sfo, C::kSfBytes, &bars->sfl[s]);
+                        bulk_load(st + 3 * kTileBytes + 2 * C::kSfBytes, gw + sfo, C::kSfBytes, &bars->sfl[s]);
+                        mbar_arrive_expect_tx(&bars->full[s], 3 * kTileBytes);
                         tma_load_2d(st, &tm_b, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
                         tma_load_2d(st + kTileBytes, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
                         tma_load_2d(st + 2 * kTileBytes, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
-                        bulk_load(st + 3 * kTileBytes, gb + sfo, C::kSfBytes, &bars->full[s]);
-                        bulk_load(st + 3 * kTileBytes + C::kSfBytes, gr + sfo, C::kSfBytes, &bars->full[s]);
-                        bulk_load(st + 3 * kTileBytes + 2 * C::kSfBytes, gw + sfo, C::kSfBytes, &bars->full[s]);
                     }
                 }
             }
@@ -412,7 +419,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t s = it % kStages;
-                if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
+                if (!mbar_wait(&bars->sfl[s], (it / kStages) & 1)) { ok = false; break; }
                 const uint8_t* sf = smem + s * kStride + (SPB ? SpStage::kSf : 3 * kTileBytes);
                 const uint32_t tcol = tmem + 2 * BN + s * kSfColsPerStage + lane_off;
                 if constexpr (SPB) {

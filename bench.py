@@ -47,7 +47,10 @@ from activation_sparsity_prep_b200 import workloads as wl  # noqa: E402
 
 METRIC = "SharQ linear eff. TFLOPS & tokens/s, % of FP4 roofline; prep kernel HBM GB/s"
 L2_FLUSH_BYTES = 512 << 20          # > 126 MB L2
-PREP_BYTES_PER_ELEM = {(0, 1): 3.125, (1, 1): 3.0625}   # (fmt, zero-filled backbone)
+# (fmt, zero-filled backbone): read X 2 + backbone codes + scales + residual
+# codes + scales; the compressed pair backbone stores K/4 code bytes and K/16
+# metadata bytes per row instead of K/2 codes
+PREP_BYTES_PER_ELEM = {(0, 1): 3.125, (1, 1): 3.0625, (1, 0): 2.875}
 
 
 def parse_args():
@@ -60,7 +63,9 @@ def parse_args():
     ap.add_argument("--M", type=int, default=None,
                     help="rows per linear (default: 2048 for llama8b, the workload's own M otherwise)")
     ap.add_argument("--fmt", default="nvfp4")
-    ap.add_argument("--nm", default="2:4", help="n:m of the backbone mask")
+    ap.add_argument("--nm", default="2:4",
+                    help="n:m of the backbone mask; 4:8p = the pair-granular 4:8 backbone, stored "
+                         "compressed for the sparse tensor-core MMA (MXFP4, RMSNorm workloads)")
     ap.add_argument("--residual", choices=["own", "shared"], default="own",
                     help="tensor scale of the NVFP4 residual: its own (default) or the backbone's")
     ap.add_argument("--fuse-mlp", action="store_true",
@@ -217,10 +222,12 @@ def profiled_traffic(launch_key: str, sha: str):
 # ------------------------------------------------------------ CPU arm ----
 
 def oracle_sample_step(linears, rows: int, quantized, fmt="nvfp4", n=2, m=4, residual="own",
-                       fuse_mlp=False):
+                       fuse_mlp=False, pairs=False):
     """One bounded oracle step: prepare and linear of the first `rows` rows
     of every linear.  fuse_mlp: the down projection's input is the SwiGLU of
     the gate+up output (rounded to bf16) instead of its synthetic tensor.
+    pairs: the pair-granular 4:8 prepare (its compressed form is only a
+    storage layout; the linear reads the same operands).
     Returns (seconds, effective flops of the sample)."""
     import oracle
     t0 = time.perf_counter()
@@ -228,8 +235,11 @@ def oracle_sample_step(linears, rows: int, quantized, fmt="nvfp4", n=2, m=4, res
     H = None
     for (L, d), Wq in zip(linears, quantized):
         X = d["X"][:rows] if not (fuse_mlp and L.name == "down") else H
-        P = oracle.prepare(X, d["gamma"], wl.EPS, n, m, fmt, residual_scale=residual,
-                           norm=d["norm"], beta=d["beta"])
+        if pairs:
+            P = oracle.prepare_pairs(X, d["gamma"], wl.EPS)[0]
+        else:
+            P = oracle.prepare(X, d["gamma"], wl.EPS, n, m, fmt, residual_scale=residual,
+                               norm=d["norm"], beta=d["beta"])
         if fuse_mlp and L.name == "gate_up":
             H = oracle.bf16_rne_from_f64(oracle.swiglu_linear(P, Wq))
         else:
@@ -341,7 +351,7 @@ def cpu_baseline(linears, args, budget_s: float = 10.0, rows: int = 16):
         total_t, total_f, n = 0.0, 0.0, 0
         while total_t < budget_s and n < 50:
             t, f = oracle_sample_step(linears, rows, quantized, args.fmt, n_, m_, args.residual,
-                                      args.fuse_mlp)
+                                      args.fuse_mlp, pairs_of(args))
             total_t += t
             total_f += f
             n += 1
@@ -361,7 +371,8 @@ def cpu_baseline(linears, args, budget_s: float = 10.0, rows: int = 16):
             "single_thread_value": one,
             "sample": f"{n} passes of: oracle prepare + fp64 two-path linear on the first {rows} "
                       f"rows of each of the {len(linears)} linears (all N"
-                      f"{'; SwiGLU of gate+up feeds down' if args.fuse_mlp else ''}); prepare "
+                      f"{'; SwiGLU of gate+up feeds down' if args.fuse_mlp else ''}"
+                      f"{'; pair-granular 4:8 prepare' if pairs_of(args) else ''}); prepare "
                       f"single-threaded C, GEMM numpy/OpenBLAS fp64 on {threads} threads "
                       f"(single_thread_value: the same sample with one BLAS thread)"}
 
@@ -379,6 +390,8 @@ def workload_desc(W, M):
 
 def bench_config(args, W, M):
     return {"workload": workload_desc(W, M), "M": M, "fmt": args.fmt, "nm": args.nm,
+            "backbone": ("pair-granular 4:8, compressed [M, K/4] + pair metadata, sparse tensor-core MMA"
+                         if pairs_of(args) else "element n:m, zero-filled [M, K/2], dense MMA"),
             "residual_scale": args.residual,
             "mlp": ("producer-fused: gate_up writes H = silu(gate)*up and max|H| (SwiGLU epilogue), "
                     "down prepares that H from the producer's amax" if args.fuse_mlp else
@@ -402,7 +415,7 @@ def run_reference(args):
                                             else d["W"], args.fmt) for L, d in linears]
         rows = 16
         step = lambda: oracle_sample_step(linears, rows, quantized, args.fmt, n, m, args.residual,
-                                          args.fuse_mlp)
+                                          args.fuse_mlp, pairs_of(args))
         what = (f"first {rows} rows of each linear per step (all N), of M={args.M}"
                 + ("; the SwiGLU of gate+up (bf16) feeds down" if args.fuse_mlp else ""))
         M = args.M
@@ -442,8 +455,13 @@ def run_reference(args):
 # ------------------------------------------------------------ GPU arm ----
 
 def nm_of(args):
-    n, m = (int(v) for v in args.nm.split(":"))
+    n, m = (int(v) for v in args.nm.rstrip("p").split(":"))
     return n, m
+
+
+def pairs_of(args) -> bool:
+    """--nm 4:8p: the pair-granular backbone on the sparse MMA."""
+    return args.nm.endswith("p")
 
 
 def build_units(args, dev):
@@ -456,6 +474,7 @@ def build_units(args, dev):
     W = wl.WORKLOADS[args.workload]
     fmt = sq._FMT[args.fmt]
     n, m = nm_of(args)
+    pairs = pairs_of(args)
     bf = torch.bfloat16
     up = lambda a: torch.from_numpy(a).view(bf).to(dev)
     units = []
@@ -472,7 +491,8 @@ def build_units(args, dev):
                 Wt = sq.interleave_gate_up(Wt[:L.N // 2], Wt[L.N // 2:])
             w = sq.quantize_weight(Wt, fmt)
             del Wt
-            P = sq.Prepared.empty(M, L.K, n, m, fmt, device=dev, residual_scale=args.residual)
+            P = sq.Prepared.empty(M, L.K, n, m, fmt, device=dev, residual_scale=args.residual,
+                                  pairs=pairs)
             ws = torch.empty(max(256, sq.prepare_workspace_bytes(M, L.K, fmt)), dtype=torch.uint8, device=dev)
             if swiglu:
                 Y = torch.empty((M, L.N // 2), dtype=bf, device=dev)
@@ -630,7 +650,9 @@ def run_sharq(args):
     # roofline time = max(flops / FP4 peak, algorithmic bytes / HBM): weight codes
     # + scales once, activation codes + scales of both paths, bf16 output
     sfb = 1.0 / (16 if fmt == 0 else 32)
-    lin_bytes = (ud["N"] * ud["K"] * (0.5 + sfb) + ud["rows"] * ud["K"] * 2 * (0.5 + sfb)
+    pairs = pairs_of(args)
+    bb_bytes = (0.25 + 1.0 / 16 + sfb) if pairs else (0.5 + sfb)     # compressed codes + metadata
+    lin_bytes = (ud["N"] * ud["K"] * (0.5 + sfb) + ud["rows"] * ud["K"] * (bb_bytes + 0.5 + sfb)
                  + 2.0 * ud["Y"].numel())
     lin_flops = alg_factor * ud["rows"] * ud["N"] * ud["K"]
     hbm_bound = lin_bytes / (hbm * 1e9) > lin_flops / (fp4_peak * 1e12)
@@ -638,15 +660,17 @@ def run_sharq(args):
         achieved, lin_peak, lin_unit = lin_bytes / lin_t[dom] / 1e9, hbm, "GB/s"
     else:
         achieved, lin_peak, lin_unit = lin_flops / lin_t[dom] / 1e12, fp4_peak, "TFLOP/s"
-    lin_key = f"linear_{args.fmt}_{args.workload}_{ud['name']}{'_swiglu' if ud.get('swiglu') else ''}_M{args.M}"
+    tag = "_pairs" if pairs else ""
+    lin_key = (f"linear_{args.fmt}{tag}_{args.workload}_{ud['name']}{'_swiglu' if ud.get('swiglu') else ''}"
+               f"_M{args.M}")
     traffic = profiled_traffic(lin_key, source_sha("linear.cu", "common.cuh"))
     # Prepare roofline on its largest launch (algorithmic bytes per element:
     # read X 2, backbone codes 0.5 (zero-filled) + scales, residual codes 0.5 + scales)
-    bpe = PREP_BYTES_PER_ELEM[(fmt, 1)]
+    bpe = PREP_BYTES_PER_ELEM[(fmt, 0 if pairs else 1)]
     pdom = max(range(len(units)), key=lambda i: prep_t[i])
     up_ = units[pdom]
     prep_ach = bpe * up_["prep_rows"] * up_["K"] / prep_t[pdom] / 1e9
-    prep_key = f"prepare_{args.fmt}_{args.workload}_{up_['name']}_M{args.M}"
+    prep_key = f"prepare_{args.fmt}{tag}_{args.workload}_{up_['name']}_M{args.M}"
     prep_traffic = profiled_traffic(prep_key, source_sha("prepare.cu", "common.cuh"))
 
     # end-to-end: host inputs (pinned) in, host outputs out, every step
@@ -700,7 +724,9 @@ def run_sharq(args):
                          "peak_note": (f"{src} copy bandwidth" if hbm_bound else
                                        f"dense FP4 = 4 x {src} bf16 burst ({bf16:.0f} TFLOP/s)"),
                          "achieved_note": f"{alg_factor:g}*M*N*K per launch ({n}:{m} backbone at 2x "
-                                          f"rate + dense residual)"},
+                                          f"rate + dense residual)"
+                                          + ("; backbone on tcgen05.mma.sp" if pairs else
+                                             "; backbone zero-filled on the dense MMA")},
             "prepare_roofline": {"bound": "hbm", "achieved": prep_ach, "peak": hbm, "unit": "GB/s",
                                  "frac": prep_ach / hbm, "traffic": prep_traffic,
                                  "kernel": f"prepare_kernel, {up_['name']} launch rows={up_['prep_rows']} "
@@ -708,7 +734,11 @@ def run_sharq(args):
                                  "bytes_per_elem": bpe, "peak_note": f"{src} copy bandwidth"},
             "kernel_ms": {u["name"]: {"prepare": statistics.mean(p), "linear": statistics.mean(l)}
                           for u, p, l in zip(units, prep_ms, lin_ms)},
-            "executed_fp4_tflops": sum(4.0 * u["rows"] * u["N"] * u["K"] for u in units) / sum(lin_t) / 1e12,
+            # dense-rate equivalent of what the tensor cores execute: both paths as
+            # dense MMAs (zero-filled backbone), or the residual dense plus the
+            # compressed backbone on the sparse MMA at twice the rate
+            "executed_fp4_tflops": sum((3.0 if pairs else 4.0) * u["rows"] * u["N"] * u["K"]
+                                       for u in units) / sum(lin_t) / 1e12,
             "prepare_gbs_all": sum(bpe * u["prep_rows"] * u["K"] for u in units) / sum(prep_t) / 1e9,
             "gpu_launches": (2 * len(units) + (len(units) if wl.WORKLOADS[args.workload].moe else 0))
                             * args.steps,
@@ -732,6 +762,11 @@ def main():
         args.M = 2048 if args.workload == "llama8b" else (Ms[0] if Ms else 0)
     if args.fuse_mlp and not mlp_fusable(wl.WORKLOADS[args.workload]):
         raise SystemExit("--fuse-mlp needs a workload with gate_up and down linears")
+    if pairs_of(args):
+        W = wl.WORKLOADS[args.workload]
+        if (args.nm != "4:8p" or args.fmt != "mxfp4" or args.fuse_mlp or W.moe is not None
+                or any(L.layernorm for L in W.linears)):
+            raise SystemExit("--nm 4:8p: MXFP4, RMSNorm (or no norm) plain linears, no --fuse-mlp")
     if args.impl == "reference":
         return run_reference(args)
     return run_sharq(args)
