@@ -46,6 +46,9 @@ constexpr int kWarps = kThreads / 32;
 // gamma / beta are staged in shared memory as fp32 up to this many bytes
 // (two CTAs per SM still fit); longer rows read them from global memory.
 constexpr int kMaxStagedBytes = 96 * 1024;
+// MXFP4 RMSNorm rows of up to 32 * kRowChunks 16-byte chunks (K <= 4096)
+// are loaded into registers whole in phase 1.
+constexpr int kRowChunks = 16;
 
 struct PrepArgs {
     const uint16_t* X;       // [M, K] bf16
@@ -585,6 +588,38 @@ prepare_kernel(PrepArgs a) {
         // loads in flight per lane.
         for (int64_t row = gwarp; row < M; row += nwarps) {
             const uint16_t* xr = a.X + row * K;
+            if constexpr (!LN && FMT == 1) {
+                if (nchunk <= 32 * kRowChunks) {
+                    // MXFP4 takes only rinv here: the whole row's chunk loads
+                    // in flight at once, then the same reduction order as
+                    // below.  (For NVFP4, which also takes max |y| here, the
+                    // register-held row costs spills and is slower than the
+                    // second pass over the row through L1.)
+                    uint4 v[kRowChunks];
+#pragma unroll
+                    for (int u = 0; u < kRowChunks; ++u)
+                        if (lane + 32 * u < nchunk) v[u] = ld_nc_v4(xr + (int64_t)(lane + 32 * u) * 8);
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < kRowChunks; ++u) {
+                        if (lane + 32 * u < nchunk) {
+                            float2 x[4];
+                            unpack_bf16x8(v[u], x);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                acc = __fadd_rn(acc, __fmul_rn(x[t].x, x[t].x));
+                                acc = __fadd_rn(acc, __fmul_rn(x[t].y, x[t].y));
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1)
+                        acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+                    const float rinv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(acc, (float)K), a.eps)));
+                    if (lane == 0) rinv_ws[row] = rinv;
+                    continue;
+                }
+            }
             auto row_sum = [&](auto f) {
                 float acc = 0.0f;
                 for (int c0 = lane; c0 < nchunk; c0 += 256) {
