@@ -634,6 +634,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
 // steps; each drains its partial (already scaled by the tensor scales)
 // into its shared memory and rank 0 sums the partials in rank order over
 // distributed shared memory before storing Y.
+// SwiGLU form (SW): with the interleaved gate+up weight, tensor-memory lanes
+// 0..63 of a tile are the gate rows and lanes 64..127 the up rows of the
+// same 64 features, i.e. epilogue warps 0-1 hold gates and 2-3 ups.  The
+// gate warps leave their values in a shared-memory slot ([NT][64] fp32,
+// two bounded mbarriers: full after the gate warps wrote it, empty after
+// the up warps read it), and the up warps write H = silu(gate) * up and
+// the running max |H|.
 // ------------------------------------------------------------------------
 template <int FMT, int NT>
 struct DecCfg {
@@ -658,6 +665,8 @@ struct alignas(8) DecBarriers {
     uint64_t sf_full[S];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t xg_full;         // SwiGLU: the gate warps wrote the gate values of a tile
+    uint64_t xg_empty;        // SwiGLU: the up warps consumed them
     uint32_t tmem_base;
 };
 
@@ -670,7 +679,7 @@ __device__ __forceinline__ void mma_id(uint32_t idesc0, uint32_t d, uint64_t a, 
     else          tc_mma_mxf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
 }
 
-template <int FMT, bool ONE, int NT>
+template <int FMT, bool ONE, int NT, bool SW = false>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_r, const uint8_t* __restrict__ sf_w,
@@ -682,6 +691,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     DecBarriers<S>* bars = reinterpret_cast<DecBarriers<S>*>(smem + S * D::kStageStride);
+    // SwiGLU: gate values of one tile, [NT tokens][64 features], after the barriers
+    float* xg = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(bars) + sizeof(DecBarriers<S>) + 15) & ~uintptr_t(15));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = K / BK;
@@ -696,6 +707,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
             mbar_init(&bars->acc_full[b], 1);
             mbar_init(&bars->acc_empty[b], 4);
         }
+        mbar_init(&bars->xg_full, 2);
+        mbar_init(&bars->xg_empty, 2);
         fence_barrier_init();
     }
     if (warp == 1) { tmem_alloc(&bars->tmem_base, kTmemCols); tmem_relinquish(); }
@@ -804,11 +817,61 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         const float gb = *ep.bb_tscale * gwv, gr = *ep.rs_tscale * gwv;
         const int rows = (int)(ep.M < NT ? ep.M : NT);
         uint32_t tc = 0;
+        uint32_t hmax = 0;
         for (int tile = tile0; tile < ntiles; tile += tstride, ++tc) {
             const uint32_t buf = tc & 1u, use = tc >> 1;
             const bool ok = mbar_wait(&bars->acc_full[buf], use & 1);
             tc_fence_after();
             if (!ok) break;
+            if (SW && split == 1) {
+                // lanes 0..63 of the tile hold gate rows (warps q = 0, 1), lanes
+                // 64..127 the up rows of the same features (q = 2, 3)
+                const uint32_t src = tmem + buf * 2 * NT + lane_off;
+                float v[NT];
+#pragma unroll
+                for (int c0 = 0; c0 < NT; c0 += 16) {
+                    uint32_t vb[16], vr[16];
+                    tmem_ld_32x32b_x16(src + c0, vb);
+                    if (!ONE) tmem_ld_32x32b_x16(src + NT + c0, vr);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        v[c0 + t] = ONE ? gb * __uint_as_float(vb[t])
+                                        : gb * __uint_as_float(vb[t]) + gr * __uint_as_float(vr[t]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+                const int j = (q & 1) * 32 + lane;              // feature within the tile
+                bool good = true;
+                if (q < 2) {
+                    if (tc > 0) good = mbar_wait(&bars->xg_empty, (tc - 1) & 1);
+                    if (good) {
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) xg[t * 64 + j] = v[t];
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->xg_full);
+                } else {
+                    good = mbar_wait(&bars->xg_full, tc & 1);
+                    if (good) {
+                        const int64_t hcol = (int64_t)tile * (BM / 2) + j;
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            if (t < rows) {
+                                const float h = __fmul_rn(silu_f32(xg[t * 64 + j]), v[t]);
+                                const __nv_bfloat16 hb = __float2bfloat16_rn(h);
+                                static_cast<__nv_bfloat16*>(ep.Y)[(int64_t)t * (ep.N / 2) + hcol] = hb;
+                                hmax = max(hmax, (uint32_t)(*reinterpret_cast<const uint16_t*>(&hb) & 0x7FFFu));
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->xg_empty);
+                }
+                if (!good) break;
+                continue;
+            }
             const uint32_t src_b = tmem + buf * 2 * NT + lane_off;
             const int64_t col = (int64_t)tile * BM + q * 32 + lane;
             const int jl = q * 32 + lane;                     // column within the tile
@@ -837,12 +900,55 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
         }
+        if (SW && split == 1 && q >= 2) {
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+            if (lane == 0 && hmax) atomicMax(ep.amax, hmax << 16);
+        }
     }
     if (split > 1) {
         // every CTA's partial is in its shared memory; rank 0 adds them in
         // rank order and stores Y, then the peers may exit
         cluster_sync_all();
-        if (krank == 0 && warp >= 2 && warp < 6) {
+        if (SW && krank == 0 && warp >= 2 && warp < 6) {
+            // gate warps sum their columns and leave them in xg, then the up
+            // warps sum theirs and write H = silu(gate) * up
+            const int q = warp & 3;
+            const int jl = q * 32 + lane, j = (q & 1) * 32 + lane;
+            const int rows = (int)(ep.M < NT ? ep.M : NT);
+            bool good = true;
+            if (q >= 2) good = mbar_wait(&bars->xg_full, 0);
+            uint32_t hmax = 0;
+            for (int t0 = 0; t0 < rows && good; t0 += 16) {
+                float y[16], v[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) y[t] = partial[(t0 + t) * BM + jl];
+                for (int r = 1; r < split; ++r) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) v[t] = ld_shared_cluster_f32(&partial[(t0 + t) * BM + jl], (uint32_t)r);
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) y[t] += v[t];
+                }
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    if (q < 2) {
+                        xg[(t0 + t) * 64 + j] = y[t];
+                    } else if (t0 + t < rows) {
+                        const float h = __fmul_rn(silu_f32(xg[(t0 + t) * 64 + j]), y[t]);
+                        const __nv_bfloat16 hb = __float2bfloat16_rn(h);
+                        static_cast<__nv_bfloat16*>(ep.Y)[(int64_t)(t0 + t) * (ep.N / 2) + (int64_t)tile0 * (BM / 2) + j] = hb;
+                        hmax = max(hmax, (uint32_t)(*reinterpret_cast<const uint16_t*>(&hb) & 0x7FFFu));
+                    }
+                }
+            }
+            __syncwarp();
+            if (q < 2 && lane == 0) mbar_arrive(&bars->xg_full);
+            if (q >= 2) {
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+                if (lane == 0 && hmax) atomicMax(ep.amax, hmax << 16);
+            }
+        } else if (krank == 0 && warp >= 2 && warp < 6) {
             const int jl = (warp & 3) * 32 + lane;
             const int64_t col = (int64_t)tile0 * BM + jl;
             const int rows = (int)(ep.M < NT ? ep.M : NT);
@@ -977,7 +1083,7 @@ cudaError_t launch_gemm(const void* bb_codes, const void* bb_scales, const void*
                                                        W_rows, sc, max_tiles, s, sms);
 }
 
-template <int FMT, bool ONE, int NT>
+template <int FMT, bool ONE, int NT, bool SW = false>
 cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     using D = DecCfg<FMT, NT>;
     CUtensorMap tb, tr, tw;
@@ -985,10 +1091,14 @@ cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
         !make_code_map(&tb, p.bb_codes, p.M, p.K / 2, NT) ||
         !make_code_map(&tr, p.rs_codes, p.M, p.K / 2, NT))
         return cudaErrorInvalidValue;
-    const size_t smem = D::S * D::kStageStride + sizeof(DecBarriers<D::S>) + 1024;
+    const size_t smem = D::S * D::kStageStride + sizeof(DecBarriers<D::S>) + 16 + (SW ? NT * 64 * 4 : 0) + 1024;
     static std::atomic<bool> done[64];
-    if (cudaError_t e = set_smem_once(done, decode_kernel<FMT, ONE, NT>, smem); e != cudaSuccess) return e;
-    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32, nullptr};
+    if (cudaError_t e = set_smem_once(done, decode_kernel<FMT, ONE, NT, SW>, smem); e != cudaSuccess) return e;
+    EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32, reinterpret_cast<uint32_t*>(p.amax)};
+    if (SW) {
+        cudaError_t e = cudaMemsetAsync(p.amax, 0, sizeof(float), s);
+        if (e != cudaSuccess) return e;
+    }
     const int ntiles = p.N / BN;
     const int nk = p.K / BK;
     // fewer tiles than SMs: clusters of `split` CTAs share a tile along K,
@@ -1008,7 +1118,7 @@ cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = split > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<FMT, ONE, NT>, tw, tb, tr,
+    return cudaLaunchKernelEx(&cfg, decode_kernel<FMT, ONE, NT, SW>, tw, tb, tr,
                               static_cast<const uint8_t*>(p.w_scales),
                               static_cast<const uint8_t*>(p.bb_scales),
                               static_cast<const uint8_t*>(p.rs_scales), p.K, ep, ntiles, split);
@@ -1016,6 +1126,9 @@ cudaError_t launch_decode_t(const LinearLaunch& p, cudaStream_t s, int sms) {
 
 template <int FMT, int NT>
 cudaError_t launch_decode_nt(const LinearLaunch& p, cudaStream_t s, int sms) {
+    if (p.swiglu)
+        return p.one_acc ? launch_decode_t<FMT, true, NT, true>(p, s, sms)
+                         : launch_decode_t<FMT, false, NT, true>(p, s, sms);
     return p.one_acc ? launch_decode_t<FMT, true, NT>(p, s, sms) : launch_decode_t<FMT, false, NT>(p, s, sms);
 }
 
@@ -1035,13 +1148,10 @@ cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
         return launch_gemm_t<1, true, false, true>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p,
                                                    p.N, sc, sc.mt_count * sc.nt_count, s, sms);
     }
-    // few rows: the swapped (weight-streaming) form; the SwiGLU epilogue
-    // exists in the row-tiled form only
-    if (!p.swiglu) {
-        if (p.M <= 16) return launch_decode_nt<FMT, 16>(p, s, sms);
-        if (p.M <= 32) return launch_decode_nt<FMT, 32>(p, s, sms);
-        if (p.M <= 64) return launch_decode_nt<FMT, 64>(p, s, sms);
-    }
+    // few rows: the swapped (weight-streaming) form
+    if (p.M <= 16) return launch_decode_nt<FMT, 16>(p, s, sms);
+    if (p.M <= 32) return launch_decode_nt<FMT, 32>(p, s, sms);
+    if (p.M <= 64) return launch_decode_nt<FMT, 64>(p, s, sms);
     Sched sc{};
     sc.mt_count = (int)((p.M + BM - 1) / BM);
     sc.nt_count = p.N / BN;

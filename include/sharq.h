@@ -213,8 +213,10 @@ SHARQ_API sharq_status sharq_linear(const sharq_prepared* x, const sharq_weight*
  *       H is bf16 [M, I] (16-byte aligned, device);
  *   *h_amax = max |H| over the whole tensor (fp32 holding a bf16 value;
  *       device pointer, 4-byte aligned, written by this call; 0 for M = 0).
- * The row-tiled kernel serves every M here (no decode form).  Errors as
- * sharq_linear; NULL h_amax is SHARQ_ERR_INVALID_ARG. */
+ * Like sharq_linear, M <= 64 runs the weight-streaming decode form (the
+ * gate and up rows of a feature meet through shared memory), larger M the
+ * row-tiled kernel.  Errors as sharq_linear; NULL h_amax is
+ * SHARQ_ERR_INVALID_ARG. */
 SHARQ_API sharq_status sharq_linear_swiglu(const sharq_prepared* x, const sharq_weight* w, void* H,
                                            float* h_amax, void* stream);
 

@@ -66,9 +66,12 @@ def check_amax(H, amax):
 
 SWIGLU_SHAPES = [
     # M, I, K, fmt, residual scale
-    (16, 64, 256, "nvfp4", "own"),       # one 128-column tile
-    (1, 128, 256, "nvfp4", "own"),       # decode-sized M runs the row-tiled kernel
-    (64, 192, 512, "nvfp4", "own"),
+    (16, 64, 256, "nvfp4", "own"),       # one 128-column tile (decode form)
+    (1, 128, 256, "nvfp4", "own"),       # decode form, two tiles
+    (64, 192, 512, "nvfp4", "own"),      # decode form, the largest token tile
+    (16, 256, 4096, "nvfp4", "own"),     # decode form, 4 tiles x 2-CTA split-K clusters
+    (32, 512, 8192, "mxfp4", "own"),     # decode form, 8 tiles x 4-CTA split-K clusters
+    (20, 256, 4096, "nvfp4", "shared"),  # decode form, split-K, one accumulator
     (129, 256, 1024, "nvfp4", "own"),
     (300, 320, 2048, "nvfp4", "own"),
     (200, 192, 1024, "mxfp4", "own"),
