@@ -720,24 +720,27 @@ prepare_kernel(PrepArgs a) {
     }
 
     // padding rows of the scale atoms carry zero scales
+    // (fewer than 128 rows: one warp a row, its lanes across the row's
+    // scale words; no division)
     {
         const int words = nsf / 4;
-        const int64_t npad = (Mpad - M) * words;
-        for (int64_t i = gwarp * 32 + lane; i < npad; i += nwarps * 32) {
-            const int64_t row = M + i / words;
-            const int s4 = (int)(i % words);
-            *reinterpret_cast<uint32_t*>(a.bb_scales + sf_off(row, s4 * 4, nsf)) = 0u;
-            if (!WEIGHT) *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, s4 * 4, nsf)) = 0u;
+        const int prow = (int)(Mpad - M);
+        for (int r = (int)gwarp; r < prow; r += (int)nwarps) {
+            const int64_t row = M + r;
+            for (int s4 = lane; s4 < words; s4 += 32) {
+                *reinterpret_cast<uint32_t*>(a.bb_scales + sf_off(row, s4 * 4, nsf)) = 0u;
+                if (!WEIGHT) *reinterpret_cast<uint32_t*>(a.rs_scales + sf_off(row, s4 * 4, nsf)) = 0u;
+            }
         }
         if (PAIRS) {
             // padding rows of the metadata atoms: pairs 0 and 1 (of zero codes)
             const int kblk = K / 256;
-            const int64_t nmeta = (Mpad - M) * kblk;
-            for (int64_t i = gwarp * 32 + lane; i < nmeta; i += nwarps * 32) {
-                const int64_t row = M + i / kblk;
-                const int kb = (int)(i % kblk);
-                *reinterpret_cast<uint4*>(a.bb_meta + ((int64_t)kb * (Mpad >> 7) + (row >> 7)) * 2048 +
-                                          (row & 127) * 16) = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+            for (int r = (int)gwarp; r < prow; r += (int)nwarps) {
+                const int64_t row = M + r;
+                for (int kb = lane; kb < kblk; kb += 32)
+                    *reinterpret_cast<uint4*>(a.bb_meta + ((int64_t)kb * (Mpad >> 7) + (row >> 7)) * 2048 +
+                                              (row & 127) * 16) =
+                        make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
             }
         }
     }
