@@ -135,9 +135,13 @@ struct TileInfo {
 
 constexpr int kMaxExperts = 256;    // keeps the scheduler's shared memory at 3 KiB
 
-// Tile scheduler.  Plain linear: m fastest, so the CTAs working at one time
-// share weight tiles (each weight tile is read from HBM about once) while
-// the activation tiles stay resident in L2.  Grouped linear: expert-major,
+// Tile scheduler.  Plain linear: the CTAs working at one time walk
+// neighbouring tiles of the fast dimension, so they share the slow
+// dimension's operand tiles, and the fast dimension's operand rows (all of
+// them) stay resident in L2 while the other operand streams from HBM about
+// once.  m fastest keeps the activations resident, n fastest the weight;
+// the launch keeps the smaller of the two resident (with the larger one
+// resident-but-too-big, it would stream from HBM once per wave of tiles).  Grouped linear: expert-major,
 // then n, then m, so one expert's weight and activation rows stay hot in L2
 // while its tiles run; rows of expert e sit at a 128-aligned padded offset
 // of the gathered operands.
@@ -150,6 +154,7 @@ struct Sched {
     int E;
     int64_t w_sf_stride;       // grouped: bytes of one expert's scale buffer
     int N;
+    int n_fast;                // plain: n-tiles fastest instead of m-tiles
 };
 
 struct SchedTables {
@@ -211,7 +216,9 @@ __device__ __forceinline__ int sched_count(const Sched& sc, const SchedSmem* sm)
 __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem* sm, int t) {
     TileInfo ti;
     if (!sc.grouped) {
-        const int nt = t / sc.mt_count, mt = t - nt * sc.mt_count;
+        int nt, mt;
+        if (sc.n_fast) { mt = t / sc.nt_count; nt = t - mt * sc.nt_count; }
+        else           { nt = t / sc.mt_count; mt = t - nt * sc.mt_count; }
         ti.a_row = (int64_t)mt * 128;
         ti.w_row = (int64_t)nt * 128;
         ti.w_sf = (int64_t)nt * (sc.nsf / 4) * 512;
@@ -1132,6 +1139,16 @@ cudaError_t launch_decode_nt(const LinearLaunch& p, cudaStream_t s, int sms) {
     return p.one_acc ? launch_decode_t<FMT, true, NT>(p, s, sms) : launch_decode_t<FMT, false, NT>(p, s, sms);
 }
 
+// Plain tile walk: n fastest when the activation operands (both paths'
+// codes and scales) outweigh the weight's, so the smaller operand is the
+// L2-resident one.
+inline int walk_n_fast(const LinearLaunch& p) {
+    const double sfb = p.fmt == 0 ? 1.0 / 16 : 1.0 / 32;
+    const double a_bytes = (double)p.M * p.K * 2.0 * (0.5 + sfb);
+    const double w_bytes = (double)p.N * p.K * (0.5 + sfb);
+    return a_bytes > w_bytes ? 1 : 0;
+}
+
 template <int FMT>
 cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     if (p.bb_meta) {
@@ -1145,6 +1162,7 @@ cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
         sc.nsf = p.K / Cfg<FMT>::BS;
         sc.grouped = 0;
         sc.N = p.N;
+        sc.n_fast = walk_n_fast(p);
         return launch_gemm_t<1, true, false, true>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p,
                                                    p.N, sc, sc.mt_count * sc.nt_count, s, sms);
     }
@@ -1159,6 +1177,7 @@ cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     sc.nsf = p.K / Cfg<FMT>::BS;
     sc.grouped = 0;
     sc.N = p.N;
+    sc.n_fast = walk_n_fast(p);
     return launch_gemm<FMT>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p, p.N, sc,
                             sc.mt_count * sc.nt_count, s, sms);
 }
