@@ -417,7 +417,8 @@ def run_reference(args):
         step = lambda: oracle_sample_step(linears, rows, quantized, args.fmt, n, m, args.residual,
                                           args.fuse_mlp, pairs_of(args))
         what = (f"first {rows} rows of each linear per step (all N), of M={args.M}"
-                + ("; the SwiGLU of gate+up (bf16) feeds down" if args.fuse_mlp else ""))
+                + ("; the SwiGLU of gate+up (bf16) feeds down" if args.fuse_mlp else "")
+                + ("; pair-granular 4:8 prepare" if pairs_of(args) else ""))
         M = args.M
     else:
         sample = moe_reference_sample(W, args.fmt, fuse_mlp=args.fuse_mlp)

@@ -59,3 +59,16 @@ def test_reference_arm_runs_the_fused_moe_layer():
     j = _run("--workload", "qwen3moe", "--fuse-mlp")
     assert j["config"]["mlp"].startswith("producer-fused") and j["value"] > 0
     assert "SwiGLU" in j["cpu_baseline"]["sample"]
+
+
+def test_reference_arm_runs_the_pair_backbone():
+    j = _run("--workload", "tiny", "--fmt", "mxfp4", "--nm", "4:8p")
+    assert j["config"]["nm"] == "4:8p" and j["config"]["backbone"].startswith("pair-granular")
+    assert "pair-granular" in j["cpu_baseline"]["sample"] and j["value"] > 0
+
+
+def test_pair_backbone_needs_mxfp4():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--nm", "4:8p", "--steps", "1", "--warmup", "0"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode != 0 and "MXFP4" in out.stderr

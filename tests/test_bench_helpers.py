@@ -59,3 +59,20 @@ def test_fused_mlp_workloads():
     assert bench.mlp_fusable(wl.WORKLOADS["llama8b"]) and bench.mlp_fusable(wl.WORKLOADS["qwen3moe"])
     assert bench.mlp_fusable(wl.WORKLOADS["tiny_mlp"])
     assert not bench.mlp_fusable(wl.WORKLOADS["tiny"]) and not bench.mlp_fusable(wl.WORKLOADS["sweep"])
+
+
+def test_prepare_bytes_per_element():
+    """Read X (bf16) + backbone codes and scales + residual codes and scales:
+    zero-filled backbones store K/2 code bytes a row, the pair backbone K/4
+    plus K/16 bytes of pair indices."""
+    assert bench.PREP_BYTES_PER_ELEM[(0, 1)] == 2 + 0.5 + 1 / 16 + 0.5 + 1 / 16
+    assert bench.PREP_BYTES_PER_ELEM[(1, 1)] == 2 + 0.5 + 1 / 32 + 0.5 + 1 / 32
+    assert bench.PREP_BYTES_PER_ELEM[(1, 0)] == 2 + 0.25 + 1 / 16 + 1 / 32 + 0.5 + 1 / 32
+
+
+def test_nm_parsing():
+    import argparse
+    a = argparse.Namespace(nm="4:8p")
+    assert bench.nm_of(a) == (4, 8) and bench.pairs_of(a)
+    a = argparse.Namespace(nm="2:4")
+    assert bench.nm_of(a) == (2, 4) and not bench.pairs_of(a)
