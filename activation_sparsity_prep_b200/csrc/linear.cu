@@ -17,10 +17,12 @@
 // a residual quantised against the backbone's tensor scale) both MMAs
 // accumulate into one accumulator, Y = G_w * G_b * acc, and the two
 // tensor-memory accumulators serve as a double buffer instead: the next
-// tile's MMAs run while the epilogue drains the previous one.  The backbone
-// runs as a dense MMA over zero-filled codes: the FP4 sparse MMA carries one
-// scale per 32 logical elements, which cannot express NVFP4's per-16
-// backbone scales.
+// tile's MMAs run while the epilogue drains the previous one.  An element
+// n:m backbone runs as a dense MMA over zero-filled codes: the FP4 sparse
+// MMA carries one scale per 32 logical elements, which cannot express
+// NVFP4's per-16 backbone scales, and its metadata selects whole pairs.  The
+// pair-granular 4:8 MXFP4 backbone, stored compressed, runs on the sparse
+// MMA (tcgen05.mma.sp) instead (SPB).
 //
 // CTA layout (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
 // and MMA issuer, warps 2..5 = epilogue (one TMEM lane quarter each),

@@ -9,6 +9,11 @@
 //   phase 2  mask, backbone codes/scales with G_b, residual r,
 //            A_r = max|r|                                 -> grid barrier
 //   phase 3  residual codes/scales with G_r
+// With the residual's own tensor scale, phase 1 also takes P, the largest
+// |y| the mask prunes (the residual of a pruned entry is y itself, so
+// A_r >= P), and phase 2 already quantises the residual against P; when
+// the residual's maximum turns out to be P exactly, those are the final
+// codes and phase 3 is skipped.
 // One persistent cooperative launch runs the three phases.  In phase 1 each
 // warp owns whole rows, lane l reading the 16-byte chunks l, l+32, ... of a
 // row, which is also the fixed fp32 reduction order of the RMS sum; without
