@@ -82,6 +82,25 @@ struct SpStage {
 static_assert(SpStage::kStride % 1024 == 0 && SpStage::kRs % 1024 == 0 && SpStage::kW % 1024 == 0,
               "swizzled tiles start on 1 KiB boundaries");
 
+// Stage of the 256-wide tile (one accumulator, 256 output columns per MMA):
+// the backbone tile (zero-filled 16 KiB, or the compressed pairs' 8 KiB),
+// the residual tile, a 256-row weight tile (32 KiB), the scale atoms of the
+// backbone rows, the residual rows and the weight's rows 0..127 and
+// 128..255, and (SPB) the pair-metadata atom.
+constexpr int BNW = 256;
+constexpr int kStagesW = 3;
+template <int FMT, bool SPB>
+struct WideStage {
+    static constexpr uint32_t kRs = SPB ? BM * (BK / 4) : kTileBytes;
+    static constexpr uint32_t kW = kRs + kTileBytes;
+    static constexpr uint32_t kSf = kW + 2 * kTileBytes;          // = the operand tiles' bytes
+    static constexpr uint32_t kSfBytes = Cfg<FMT>::kSfBytes;
+    static constexpr uint32_t kMeta = kSf + 4 * kSfBytes;
+    static constexpr uint32_t kBytes = kMeta + (SPB ? BM * 16 : 0);
+    static constexpr uint32_t kStride = (kBytes + 1023) / 1024 * 1024;
+    static_assert(kRs % 1024 == 0 && kW % 1024 == 0, "swizzled tiles start on 1 KiB boundaries");
+};
+
 struct alignas(8) Barriers {
     uint64_t full[kStages];       // the stage's operand tiles have landed
     uint64_t sfl[kStages];        // the stage's scale atoms (and pair indices) have landed
@@ -96,10 +115,15 @@ struct alignas(8) Barriers {
 // per MMA k-step for MXFP4): it goes into the instruction descriptor's
 // A/B scale-factor ID fields (bits 29-30 and 4-5) and into the top two bits
 // of the tensor-memory scale addresses.
-template <int FMT>
+// N at bits 17..22 of an instruction descriptor (N >> 3)
+constexpr uint32_t with_n(uint32_t idesc, int n) {
+    return (idesc & ~(0x3Fu << 17)) | ((uint32_t)(n >> 3) << 17);
+}
+
+template <int FMT, int TN = BN>
 __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
                                     uint32_t sfb, uint32_t acc, uint32_t sf_id) {
-    const uint32_t idesc = Cfg<FMT>::kIdesc | (sf_id << 29) | (sf_id << 4);
+    const uint32_t idesc = with_n(Cfg<FMT>::kIdesc, TN) | (sf_id << 29) | (sf_id << 4);
     const uint32_t hi = sf_id << 30;
     if (FMT == 0) tc_mma_nvf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
     else          tc_mma_mxf4(d, a, b, idesc, sfa | hi, sfb | hi, acc);
@@ -157,6 +181,7 @@ struct Sched {
     int64_t w_sf_stride;       // grouped: bytes of one expert's scale buffer
     int N;
     int n_fast;                // plain: n-tiles fastest instead of m-tiles
+    int bn;                    // plain: output columns per tile (128, or 256 for the wide tile)
 };
 
 struct SchedTables {
@@ -222,11 +247,11 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
         if (sc.n_fast) { mt = t / sc.nt_count; nt = t - mt * sc.nt_count; }
         else           { nt = t / sc.mt_count; mt = t - nt * sc.mt_count; }
         ti.a_row = (int64_t)mt * 128;
-        ti.w_row = (int64_t)nt * 128;
-        ti.w_sf = (int64_t)nt * (sc.nsf / 4) * 512;
+        ti.w_row = (int64_t)nt * sc.bn;
+        ti.w_sf = (int64_t)nt * (sc.bn / 128) * (sc.nsf / 4) * 512;
         ti.y_row = ti.a_row;
         ti.rows = (int)(sc.M - ti.a_row < 128 ? sc.M - ti.a_row : 128);
-        ti.col = nt * 128;
+        ti.col = nt * sc.bn;
         ti.e = 0;
         return ti;
     }
@@ -259,18 +284,32 @@ __device__ __forceinline__ TileInfo sched_tile(const Sched& sc, const SchedSmem*
 // per k-step two sparse MMAs (128 logical K each, pair indices in tensor
 // memory) on the backbone and four dense MMAs on the residual, all into one
 // accumulator and all on the same weight tile.
-template <int FMT, bool ONE, bool SW, bool SPB>
+// WIDE (one accumulator only): 128 x 256 output tiles.  Every MMA is 256
+// columns wide, so per unit of MMA work a k-step moves a third fewer operand
+// and scale bytes; the 256-column accumulator fills half of tensor memory,
+// so it is not double-buffered (the next tile's MMAs wait for the drain),
+// and the ring has three stages.  In tensor memory the weight's scales for
+// a 256-row tile take 8 columns per scale atom along K: the atom of rows
+// 0..127 in the first four, that of rows 128..255 in the next four (one
+// column per 32-row group, as for 128 rows).
+template <int FMT, bool ONE, bool SW, bool SPB, bool WIDE = false>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_r,
               const __grid_constant__ CUtensorMap tm_w, const uint8_t* __restrict__ sf_b,
               const uint8_t* __restrict__ sf_r, const uint8_t* __restrict__ sf_w,
               const uint8_t* __restrict__ meta, int K, EpiArgs ep, Sched sc) {
     using C = Cfg<FMT>;
+    using WS = WideStage<FMT, SPB>;
     static_assert(!SPB || (FMT == 1 && ONE && !SW), "sparse backbone: MXFP4, one accumulator");
-    constexpr uint32_t kStride = SPB ? SpStage::kStride : C::kStageStride;
+    static_assert(!WIDE || (ONE && !SW), "wide tile: one accumulator, plain epilogue");
+    constexpr int TBN = WIDE ? BNW : BN;                  // output columns per tile
+    constexpr int NST = WIDE ? kStagesW : kStages;        // pipeline stages
+    constexpr bool DBUF = ONE && !WIDE;                   // double-buffered accumulator
+    constexpr uint32_t kAccCols = WIDE ? BNW : 2 * BN;
+    constexpr uint32_t kStride = WIDE ? WS::kStride : SPB ? SpStage::kStride : C::kStageStride;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Barriers* bars = reinterpret_cast<Barriers*>(smem + kStages * kStride);
+    Barriers* bars = reinterpret_cast<Barriers*>(smem + NST * kStride);
     // 128-byte aligned: the staging buffers take 16-byte vector stores
     SchedSmem* ssm = reinterpret_cast<SchedSmem*>(
         (reinterpret_cast<uintptr_t>(bars) + sizeof(Barriers) + 127) & ~uintptr_t(127));
@@ -306,9 +345,12 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
     // that the block-scaled MMA reads.  Copying them with tcgen05.cp would
     // put 3 * kAtoms copies per stage into the MMA issue stream, where they
     // do not overlap the MMAs.
-    constexpr uint32_t kScaleCols = 3 * 4 * C::kAtoms;
+    // Per stage: the backbone's and the residual's scales (4 columns per
+    // atom each), the weight's (4, or 8 for the wide tile), the pair indices.
+    constexpr uint32_t kSfbAtomCols = WIDE ? 8 : 4;
+    constexpr uint32_t kScaleCols = (8 + kSfbAtomCols) * C::kAtoms;
     constexpr uint32_t kSfColsPerStage = kScaleCols + (SPB ? 4 : 0);   // + the pair indices
-    static_assert(2 * BN + kStages * kSfColsPerStage <= kTmemCols, "tensor memory budget");
+    static_assert(kAccCols + NST * kSfColsPerStage <= kTmemCols, "tensor memory budget");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -321,14 +363,31 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                 const uint8_t* gr = sf_r + (ti.a_row >> 7) * (nsf / 4) * 512;
                 const uint8_t* gw = sf_w + ti.w_sf;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const uint32_t s = it % kStages;
-                    if (it >= kStages && !mbar_wait(&bars->empty[s], ((it / kStages) - 1) & 1)) { ok = false; break; }
+                    const uint32_t s = it % NST;
+                    if (it >= (uint32_t)NST && !mbar_wait(&bars->empty[s], ((it / NST) - 1) & 1)) { ok = false; break; }
                     uint8_t* st = smem + s * kStride;
                     const int64_t sfo = (int64_t)kb * C::kAtoms * 512;
                     // The scale bytes come first, on their own barrier, so the
                     // scale warps stage them into tensor memory while the
                     // operand tiles are still arriving.
-                    if constexpr (SPB) {
+                    if constexpr (WIDE) {
+                        mbar_arrive_expect_tx(&bars->sfl[s], WS::kBytes - WS::kSf);
+                        bulk_load(st + WS::kSf, gb + sfo, WS::kSfBytes, &bars->sfl[s]);
+                        bulk_load(st + WS::kSf + WS::kSfBytes, gr + sfo, WS::kSfBytes, &bars->sfl[s]);
+                        // the weight's rows 0..127 and 128..255: consecutive row blocks
+                        bulk_load(st + WS::kSf + 2 * WS::kSfBytes, gw + sfo, WS::kSfBytes, &bars->sfl[s]);
+                        bulk_load(st + WS::kSf + 3 * WS::kSfBytes, gw + (int64_t)(nsf / 4) * 512 + sfo,
+                                  WS::kSfBytes, &bars->sfl[s]);
+                        if constexpr (SPB) {
+                            const int64_t mpad = (sc.M + 127) / 128 * 128;
+                            bulk_load(st + WS::kMeta, meta + ((int64_t)kb * (mpad >> 7) + (ti.a_row >> 7)) * 2048,
+                                      BM * 16, &bars->sfl[s]);
+                        }
+                        mbar_arrive_expect_tx(&bars->full[s], WS::kSf);
+                        tma_load_2d(st, &tm_b, &bars->full[s], kb * (SPB ? BK / 4 : BK / 2), (int)ti.a_row);
+                        tma_load_2d(st + WS::kRs, &tm_r, &bars->full[s], kb * (BK / 2), (int)ti.a_row);
+                        tma_load_2d(st + WS::kW, &tm_w, &bars->full[s], kb * (BK / 2), (int)ti.w_row);
+                    } else if constexpr (SPB) {
                         using P = SpStage;
                         mbar_arrive_expect_tx(&bars->sfl[s], P::kBytes - P::kSf);
                         bulk_load(st + P::kSf, gb + sfo, P::kSfBytes, &bars->sfl[s]);
@@ -361,25 +420,26 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
                 // the epilogue must have drained this buffer's previous tile
-                const uint32_t buf = ONE ? (tc & 1u) : 0u;
-                const uint32_t use = ONE ? (tc >> 1) : tc;
+                const uint32_t buf = DBUF ? (tc & 1u) : 0u;
+                const uint32_t use = DBUF ? (tc >> 1) : tc;
                 if (use > 0 && !mbar_wait(&bars->acc_empty[buf], (use - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_b = ONE ? tmem + buf * BN : t_acc_b;
                 const uint32_t d_r = ONE ? d_b : t_acc_r;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const uint32_t s = it % kStages;
-                    if (!mbar_wait(&bars->full[s], (it / kStages) & 1)) { ok = false; break; }
-                    if (!mbar_wait(&bars->sf_full[s], (it / kStages) & 1)) { ok = false; break; }
+                    const uint32_t s = it % NST;
+                    if (!mbar_wait(&bars->full[s], (it / NST) & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars->sf_full[s], (it / NST) & 1)) { ok = false; break; }
                     tc_fence_after();
                     uint8_t* st = smem + s * kStride;
-                    const uint32_t t_sfa_b = tmem + 2 * BN + s * kSfColsPerStage;
+                    const uint32_t t_sfa_b = tmem + kAccCols + s * kSfColsPerStage;
                     const uint32_t t_sfa_r = t_sfa_b + 4 * C::kAtoms;
                     const uint32_t t_sfb = t_sfa_r + 4 * C::kAtoms;
                     if constexpr (SPB) {
                         using P = SpStage;
-                        const uint32_t a_bc = smem_u32(st + P::kBc), a_r = smem_u32(st + P::kRs);
-                        const uint32_t a_w = smem_u32(st + P::kW);
+                        const uint32_t a_bc = smem_u32(st + P::kBc);
+                        const uint32_t a_r = smem_u32(st + (WIDE ? WS::kRs : P::kRs));
+                        const uint32_t a_w = smem_u32(st + (WIDE ? WS::kW : P::kW));
                         const uint32_t t_meta = t_sfa_b + kScaleCols;
                         // backbone: two sparse MMAs of 128 logical K (32 stored
                         // bytes of A, 64 bytes of B per row; scale atom h holds
@@ -387,32 +447,32 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
 #pragma unroll
                         for (int h = 0; h < 2; ++h)
                             tc_mma_sp_nvf4(d_b, sdesc_sw64(a_bc + 32 * h), sdesc_sw128(a_w + 64 * h),
-                                           t_meta + 2 * h, P::kIdesc, t_sfa_b + 4 * h, t_sfb + 4 * h,
-                                           (kb | h) ? 1u : 0u);
+                                           t_meta + 2 * h, with_n(P::kIdesc, TBN), t_sfa_b + 4 * h,
+                                           t_sfb + kSfbAtomCols * h, (kb | h) ? 1u : 0u);
                         // residual: four dense MMAs of 64 K on the same weight tile
 #pragma unroll
                         for (int j = 0; j < BK / 64; ++j) {
                             const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
-                            mma<FMT>(d_r, sdesc_sw128(a_r + 32 * j), sdesc_sw128(a_w + 32 * j),
-                                     t_sfa_r + 4 * (j / C::kStepsPerAtom), t_sfb + 4 * (j / C::kStepsPerAtom),
-                                     1u, sf_id);
+                            mma<FMT, TBN>(d_r, sdesc_sw128(a_r + 32 * j), sdesc_sw128(a_w + 32 * j),
+                                          t_sfa_r + 4 * (j / C::kStepsPerAtom),
+                                          t_sfb + kSfbAtomCols * (j / C::kStepsPerAtom), 1u, sf_id);
                         }
                         tc_commit(&bars->empty[s]);
                         continue;
                     }
-                    const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + kTileBytes);
-                    const uint32_t a_w = smem_u32(st + 2 * kTileBytes);
+                    const uint32_t a_b = smem_u32(st), a_r = smem_u32(st + (WIDE ? WS::kRs : kTileBytes));
+                    const uint32_t a_w = smem_u32(st + (WIDE ? WS::kW : 2 * kTileBytes));
 #pragma unroll
                     for (int j = 0; j < BK / 64; ++j) {
                         const int at = j / C::kStepsPerAtom;
                         const uint32_t sf_id = (uint32_t)(j % C::kStepsPerAtom) * (4 / C::kStepsPerAtom);
-                        const uint32_t col = 4 * at;
+                        const uint32_t col = 4 * at, colb = kSfbAtomCols * at;
                         const uint64_t db = sdesc_sw128(a_w + 32 * j);
                         const uint32_t acc = (kb | j) ? 1u : 0u;
-                        mma<FMT>(d_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + col,
-                                 acc, sf_id);
-                        mma<FMT>(d_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + col,
-                                 ONE ? 1u : acc, sf_id);
+                        mma<FMT, TBN>(d_b, sdesc_sw128(a_b + 32 * j), db, t_sfa_b + col, t_sfb + colb,
+                                      acc, sf_id);
+                        mma<FMT, TBN>(d_r, sdesc_sw128(a_r + 32 * j), db, t_sfa_r + col, t_sfb + colb,
+                                      ONE ? 1u : acc, sf_id);
                     }
                     tc_commit(&bars->empty[s]);
                 }
@@ -427,20 +487,36 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nk; ++kb, ++it) {
-                const uint32_t s = it % kStages;
-                if (!mbar_wait(&bars->sfl[s], (it / kStages) & 1)) { ok = false; break; }
-                const uint8_t* sf = smem + s * kStride + (SPB ? SpStage::kSf : 3 * kTileBytes);
-                const uint32_t tcol = tmem + 2 * BN + s * kSfColsPerStage + lane_off;
+                const uint32_t s = it % NST;
+                if (!mbar_wait(&bars->sfl[s], (it / NST) & 1)) { ok = false; break; }
+                const uint8_t* sf = smem + s * kStride + (WIDE ? WS::kSf : SPB ? SpStage::kSf : 3 * kTileBytes);
+                const uint32_t tcol = tmem + kAccCols + s * kSfColsPerStage + lane_off;
                 if constexpr (SPB) {
                     // pair indices: tensor-memory lane r holds row r's 16 bytes
                     // of the stage in K order (four columns)
-                    const uint8_t* mt = smem + s * kStride + SpStage::kMeta;
+                    const uint8_t* mt = smem + s * kStride + (WIDE ? WS::kMeta : SpStage::kMeta);
                     tmem_st_32x32b_x4(tcol + kScaleCols, ld_shared_v4(mt + 16 * ((warp & 3) * 32 + lane)));
+                }
+                if constexpr (WIDE) {
+                    // the weight's 256 rows: per atom along K, the row block
+                    // 0..127 then 128..255, 8 consecutive columns
+                    uint4 v[2 * C::kAtoms];
+#pragma unroll
+                    for (int at = 0; at < C::kAtoms; ++at) {
+                        v[2 * at] = ld_shared_v4(sf + 2 * C::kSfBytes + 512 * at + 16 * lane);
+                        v[2 * at + 1] = ld_shared_v4(sf + 3 * C::kSfBytes + 512 * at + 16 * lane);
+                    }
+                    const uint32_t tb = tcol + 2 * 4 * C::kAtoms;
+#pragma unroll
+                    for (int h = 0; h < C::kAtoms / 2; ++h) {
+                        const uint4 w4[4] = {v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]};
+                        tmem_st_32x32b_x16(tb + 16 * h, w4);
+                    }
                 }
                 // one store per operand: its kAtoms atoms are 4 * kAtoms
                 // consecutive columns
 #pragma unroll
-                for (int o = 0; o < 3; ++o) {
+                for (int o = 0; o < (WIDE ? 2 : 3); ++o) {
                     uint4 v[C::kAtoms];
 #pragma unroll
                     for (int at = 0; at < C::kAtoms; ++at)
@@ -468,8 +544,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             const int r_local = q * 32 + lane;
             const int64_t row = ti.y_row + r_local;
             const bool row_ok = r_local < ti.rows;
-            const uint32_t buf = ONE ? (tc & 1u) : 0u;
-            const uint32_t use = ONE ? (tc >> 1) : tc;
+            const uint32_t buf = DBUF ? (tc & 1u) : 0u;
+            const uint32_t use = DBUF ? (tc >> 1) : tc;
             const bool ok = mbar_wait(&bars->acc_full[buf], use & 1);
             tc_fence_after();
             if (!ok) break;
@@ -477,7 +553,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             const int64_t col0 = ti.col;
             if (!SW && ep.y_fp32) {
 #pragma unroll 1
-                for (int cc = 0; cc < BN / 32; ++cc) {
+                for (int cc = 0; cc < TBN / 32; ++cc) {
                     uint32_t vb[32], vr[32];
                     tmem_ld_32x32b_x32(src_b + lane_off + cc * 32, vb);
                     if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
@@ -501,7 +577,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
             } else {
                 // drain the accumulators into packed bf16x2 registers (64 for
                 // Y, 32 for H), hand the tensor memory back, then store
-                constexpr int kOutCols = SW ? BN / 2 : BN;
+                constexpr int kOutCols = SW ? BN / 2 : TBN;
                 uint32_t out[kOutCols / 2];
                 if constexpr (SW) {
                     // columns j and 64 + j of the tile: gate and up of feature j,
@@ -543,7 +619,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ 
                     }
                 } else {
 #pragma unroll
-                    for (int cc = 0; cc < BN / 32; ++cc) {
+                    for (int cc = 0; cc < TBN / 32; ++cc) {
                         uint32_t vb[32], vr[32];
                         tmem_ld_32x32b_x32(src_b + lane_off + cc * 32, vb);
                         if (!ONE) tmem_ld_32x32b_x32(t_acc_r + lane_off + cc * 32, vr);
@@ -1038,21 +1114,21 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_b
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT, bool SPB = false>
+template <int FMT, bool SPB = false, bool WIDE = false>
 size_t linear_smem_bytes() {
-    const size_t stride = SPB ? SpStage::kStride : Cfg<FMT>::kStageStride;
-    return kStages * stride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
+    const size_t stride = WIDE ? WideStage<FMT, SPB>::kStride : SPB ? SpStage::kStride : Cfg<FMT>::kStageStride;
+    return (WIDE ? kStagesW : kStages) * stride + sizeof(Barriers) + 128 + sizeof(SchedSmem) + 1024;
 }
 
-template <int FMT, bool ONE, bool SW, bool SPB = false>
+template <int FMT, bool ONE, bool SW, bool SPB = false, bool WIDE = false>
 cudaError_t ensure_smem_attr() {
     static std::atomic<bool> done[64];
-    return set_smem_once(done, linear_kernel<FMT, ONE, SW, SPB>, linear_smem_bytes<FMT, SPB>());
+    return set_smem_once(done, linear_kernel<FMT, ONE, SW, SPB, WIDE>, linear_smem_bytes<FMT, SPB, WIDE>());
 }
 
 // A_rows: rows of the activation operands (gathered and padded for the
 // grouped form); W_rows: rows of the (stacked) weight.
-template <int FMT, bool ONE, bool SW, bool SPB = false>
+template <int FMT, bool ONE, bool SW, bool SPB = false, bool WIDE = false>
 cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const void* rs_codes,
                         const void* rs_scales, int64_t A_rows, const LinearLaunch& p, int64_t W_rows,
                         const Sched& sc, int max_tiles, cudaStream_t s, int sms) {
@@ -1060,9 +1136,9 @@ cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const voi
     // the compressed backbone has K/4 bytes a row: 64 bytes a k-step
     if (!make_code_map(&tb, bb_codes, A_rows, SPB ? p.K / 4 : p.K / 2, BM, SPB ? 64 : 128) ||
         !make_code_map(&tr, rs_codes, A_rows, p.K / 2, BM) ||
-        !make_code_map(&tw, p.w_codes, W_rows, p.K / 2, BN))
+        !make_code_map(&tw, p.w_codes, W_rows, p.K / 2, WIDE ? BNW : BN))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem_attr<FMT, ONE, SW, SPB>();
+    cudaError_t e = ensure_smem_attr<FMT, ONE, SW, SPB, WIDE>();
     if (e != cudaSuccess) return e;
     EpiArgs ep{p.bb_tscale, p.rs_tscale, p.w_tscale, p.Y, p.M, p.N, p.y_fp32,
                reinterpret_cast<uint32_t*>(p.amax)};
@@ -1071,7 +1147,7 @@ cudaError_t launch_gemm_t(const void* bb_codes, const void* bb_scales, const voi
         if (e != cudaSuccess) return e;
     }
     const int grid = std::max(1, std::min(max_tiles, std::max(1, sms)));
-    linear_kernel<FMT, ONE, SW, SPB><<<grid, kThreads, linear_smem_bytes<FMT, SPB>(), s>>>(
+    linear_kernel<FMT, ONE, SW, SPB, WIDE><<<grid, kThreads, linear_smem_bytes<FMT, SPB, WIDE>(), s>>>(
         tb, tr, tw, static_cast<const uint8_t*>(bb_scales), static_cast<const uint8_t*>(rs_scales),
         static_cast<const uint8_t*>(p.w_scales), static_cast<const uint8_t*>(p.bb_meta), p.K, ep, sc);
     return cudaGetLastError();
@@ -1151,20 +1227,44 @@ inline int walk_n_fast(const LinearLaunch& p) {
     return a_bytes > w_bytes ? 1 : 0;
 }
 
+// The 256-wide tile (one accumulator only) moves a third fewer operand and
+// scale bytes per unit of MMA work, but has one accumulator buffer and half
+// as many tiles: it is taken where its last wave over the SMs is not much
+// emptier than the 128-wide tile's.
+inline bool use_wide(const LinearLaunch& p, int sms) {
+    if (!p.one_acc || p.swiglu || p.N % BNW != 0) return false;
+    const int64_t g = std::max(1, sms);
+    const int64_t mt = (p.M + BM - 1) / BM;
+    auto fill = [g](int64_t tiles) { return (double)tiles / (double)(((tiles + g - 1) / g) * g); };
+    return fill(mt * (p.N / BNW)) * 1.1 >= fill(mt * (p.N / BN));
+}
+
+inline Sched plain_sched(const LinearLaunch& p, int bn, int nsf) {
+    Sched sc{};
+    sc.mt_count = (int)((p.M + BM - 1) / BM);
+    sc.nt_count = p.N / bn;
+    sc.M = p.M;
+    sc.nsf = nsf;
+    sc.grouped = 0;
+    sc.N = p.N;
+    sc.n_fast = walk_n_fast(p);
+    sc.bn = bn;
+    return sc;
+}
+
 template <int FMT>
 cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
+    const int nsf = p.K / Cfg<FMT>::BS;
     if (p.bb_meta) {
         // compressed pair-granular backbone: the row-tiled kernel with the
         // sparse MMA (the swapped decode form would need the backbone as B)
         if (FMT != 1 || !p.one_acc || p.swiglu) return cudaErrorNotSupported;
-        Sched sc{};
-        sc.mt_count = (int)((p.M + BM - 1) / BM);
-        sc.nt_count = p.N / BN;
-        sc.M = p.M;
-        sc.nsf = p.K / Cfg<FMT>::BS;
-        sc.grouped = 0;
-        sc.N = p.N;
-        sc.n_fast = walk_n_fast(p);
+        if (use_wide(p, sms)) {
+            const Sched sc = plain_sched(p, BNW, nsf);
+            return launch_gemm_t<1, true, false, true, true>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales,
+                                                             p.M, p, p.N, sc, sc.mt_count * sc.nt_count, s, sms);
+        }
+        const Sched sc = plain_sched(p, BN, nsf);
         return launch_gemm_t<1, true, false, true>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p,
                                                    p.N, sc, sc.mt_count * sc.nt_count, s, sms);
     }
@@ -1172,14 +1272,12 @@ cudaError_t launch_linear_t(const LinearLaunch& p, cudaStream_t s, int sms) {
     if (p.M <= 16) return launch_decode_nt<FMT, 16>(p, s, sms);
     if (p.M <= 32) return launch_decode_nt<FMT, 32>(p, s, sms);
     if (p.M <= 64) return launch_decode_nt<FMT, 64>(p, s, sms);
-    Sched sc{};
-    sc.mt_count = (int)((p.M + BM - 1) / BM);
-    sc.nt_count = p.N / BN;
-    sc.M = p.M;
-    sc.nsf = p.K / Cfg<FMT>::BS;
-    sc.grouped = 0;
-    sc.N = p.N;
-    sc.n_fast = walk_n_fast(p);
+    if (use_wide(p, sms)) {
+        const Sched sc = plain_sched(p, BNW, nsf);
+        return launch_gemm_t<FMT, true, false, false, true>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales,
+                                                            p.M, p, p.N, sc, sc.mt_count * sc.nt_count, s, sms);
+    }
+    const Sched sc = plain_sched(p, BN, nsf);
     return launch_gemm<FMT>(p.bb_codes, p.bb_scales, p.rs_codes, p.rs_scales, p.M, p, p.N, sc,
                             sc.mt_count * sc.nt_count, s, sms);
 }

@@ -107,6 +107,8 @@ SHAPES = [
     (1, 1024, 4096, "mxfp4"),
     # K long enough that clusters of 4 and 8 CTAs split each tile along K
     (5, 256, 8192, "nvfp4"),
+    # the 256-wide tile (one accumulator, enough tiles to fill the SMs), ragged M
+    (1000, 4608, 1024, "mxfp4"),
     (1, 128, 16384, "nvfp4"),
 ]
 
@@ -185,7 +187,8 @@ def test_linear_full_size_llama_prefill_sampled(lin):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("M,N,K,gk", [(16, 256, 256, "ones"), (300, 512, 4096, "ones"),
-                                      (129, 384, 1024, None), (2048, 1024, 4096, "random")])
+                                      (129, 384, 1024, None), (2048, 1024, 4096, "random"),
+                                      (1024, 4608, 1024, "ones")])     # the 256-wide tile
 def test_linear_shared_residual_scale(M, N, K, gk):
     """GPU prepare (shared) bit-exact against the oracle, then the
     single-accumulator linear against the fp64 two-path product."""

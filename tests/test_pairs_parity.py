@@ -112,6 +112,7 @@ LINEAR_CASES = [
     (129, 384, 1024),
     (300, 512, 2048),
     (2048, 1024, 4096),
+    (1000, 4608, 2048),     # the 256-wide tile, ragged M
 ]
 
 
