@@ -465,6 +465,12 @@ def pairs_of(args) -> bool:
     return args.nm.endswith("p")
 
 
+def traffic_tag(args) -> str:
+    """Part of a profiles/traffic.json key that names the kernel form."""
+    return (("_pairs" if pairs_of(args) else "") + ("_shared" if args.residual == "shared" else "")
+            + ("_fused" if args.fuse_mlp else ""))
+
+
 def build_units(args, dev):
     """Device buffers and closures for one step of the chosen workload.
     A unit is one prepare followed by one (plain or grouped) linear."""
@@ -661,7 +667,9 @@ def run_sharq(args):
         achieved, lin_peak, lin_unit = lin_bytes / lin_t[dom] / 1e9, hbm, "GB/s"
     else:
         achieved, lin_peak, lin_unit = lin_flops / lin_t[dom] / 1e12, fp4_peak, "TFLOP/s"
-    tag = "_pairs" if pairs else ""
+    # the key names the kernel form: the pair backbone and the shared residual
+    # scale run other instances (and the shared scale the 256-wide tile)
+    tag = traffic_tag(args)
     lin_key = (f"linear_{args.fmt}{tag}_{args.workload}_{ud['name']}{'_swiglu' if ud.get('swiglu') else ''}"
                f"_M{args.M}")
     traffic = profiled_traffic(lin_key, source_sha("linear.cu", "common.cuh"))

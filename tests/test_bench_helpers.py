@@ -76,3 +76,15 @@ def test_nm_parsing():
     assert bench.nm_of(a) == (4, 8) and bench.pairs_of(a)
     a = argparse.Namespace(nm="2:4")
     assert bench.nm_of(a) == (2, 4) and not bench.pairs_of(a)
+
+
+def test_traffic_key_names_the_kernel_form():
+    """A capture of the own-scale launch must not be reported for the shared
+    residual scale or the pair backbone, which run other kernel instances."""
+    import argparse
+    ns = lambda nm="2:4", residual="own", fuse_mlp=False: argparse.Namespace(nm=nm, residual=residual,
+                                                                            fuse_mlp=fuse_mlp)
+    assert bench.traffic_tag(ns()) == ""
+    assert bench.traffic_tag(ns(residual="shared")) == "_shared"
+    assert bench.traffic_tag(ns(nm="4:8p")) == "_pairs"
+    assert bench.traffic_tag(ns(fuse_mlp=True)) == "_fused"
