@@ -143,8 +143,9 @@ uint8_t orc_mx_scale_code(float amax) {
 /*   ms = S / K; rinv = 1 / sqrt(ms + eps); y_k = (x_k * rinv) * gamma_k.    */
 /* The pages say only that normalisation is fused into the preparation       */
 /* operator (Abstract); RMSNorm and the order are this library's reading.    */
-/* Pinned: constant-row closed form and fp64 agreement; the bit pattern of   */
-/* the sum beyond the order definition is parity unpinned.                   */
+/* Pinned: constant-row closed form, fp64 agreement, a lane-order probe     */
+/* that only this order predicts, and bit equality with an exact-rational   */
+/* model of IEEE binary32 round-to-nearest-even evaluated in this order.    */
 /* ------------------------------------------------------------------------ */
 
 float orc_rms_rinv(const uint16_t* x_bf16, int K, float eps) {
@@ -186,7 +187,8 @@ static inline float bf16f(uint16_t b) {
 /*   rstd = 1 / sqrt(var + eps);  y_k = (d_k * rstd) * gamma_k [+ beta_k].   */
 /* Two passes (mean, then centred squares): the textbook stable form.        */
 /* Pinned: constant row (y = beta exactly), a +-a row against its closed     */
-/* form, and a lane-order probe on S1.                                       */
+/* form, a lane-order probe on S1, and bit equality of mu, rstd and y with  */
+/* an exact-rational IEEE binary32 model evaluated in this order.           */
 /* ------------------------------------------------------------------------ */
 
 static float canonical_sum(const float* v, int K) {

@@ -150,6 +150,23 @@ def test_rmsnorm_outputs_are_the_exact_fp32_model():
         assert [Fraction(float(v)) for v in y[i]] == want
 
 
+@pytest.mark.parametrize("with_beta", [False, True])
+def test_layernorm_outputs_are_the_exact_fp32_model(with_beta):
+    """y = fl(fl(fl(x - mu) * rstd) * gamma), then fl(. + beta) only when a
+    bias is given, on the model's own mu and rstd."""
+    K = 256
+    X = wl.activation("student_t", 98, 0, 2, K)
+    g = wl.gamma_random(98, 0, K)
+    b = wl.beta_random(98, 0, K) if with_beta else None
+    y = oracle.normalize_ln(X, g, b, 1e-6)
+    for i, row in enumerate(X):
+        mu, rstd = model_ln(row, 1e-6)
+        want = [rne32(rne32(rne32(bf16(x) - mu) * rstd) * bf16(gk)) for x, gk in zip(row, g)]
+        if with_beta:
+            want = [rne32(w + bf16(bk)) for w, bk in zip(want, b)]
+        assert [Fraction(float(v)) for v in y[i]] == want
+
+
 def test_the_model_sees_a_different_order():
     """A plain left-to-right sum (a plausible mistake) gives other bits than
     the oracle on at least one of these rows, so the pins above constrain
@@ -281,3 +298,125 @@ def test_mxfp4_prepare_chain_is_the_exact_model():
         assert pack(out_codes) == R.bb.codes[i].tolist()
         assert out_scales == R.bb.scales[i].tolist()
     assert float(R.bb.tscale) == 1.0
+
+
+def model_mxfp4(Y):
+    """Element codes and E8M0 block exponents of rows of exact values:
+    exponent floor(log2 amax) - 2 + 127 (clamped at 0; 0 for an all-zero
+    block), element code E2M1(v * 2^(127 - e)) -- a power-of-two scaling,
+    exact -- and the dequantised values val(code) * 2^(e - 127)."""
+    codes, scales, deq = [], [], []
+    for row in Y:
+        rc, rs, rd = [], [], []
+        for b0 in range(0, len(row), 32):
+            blk = row[b0:b0 + 32]
+            amax = max(abs(v) for v in blk)
+            e = 0
+            if amax:
+                fl = amax.numerator.bit_length() - amax.denominator.bit_length()
+                if TWO ** fl > amax:
+                    fl -= 1
+                e = max(fl - 2 + 127, 0)
+            rs.append(e)
+            for v in blk:
+                c = e2m1_code(v * TWO ** (127 - e), v < 0)
+                rc.append(c)
+                rd.append((-1 if c & 8 else 1) * E2M1[c & 7] * TWO ** (e - 127))
+        codes.append(rc)
+        scales.append(rs)
+        deq.append(rd)
+    return codes, scales, deq
+
+
+def test_mxfp4_residual_chain_is_the_exact_model():
+    """MXFP4 residual: r = fl(y - D_b) with D_b the exact dequantised
+    backbone, then r's own MXFP4 codes and exponents."""
+    M, K = 3, 256
+    X = wl.activation("laplace_outlier", 100, 0, M, K)
+    R = oracle.prepare(X, None, 1e-6, 2, 4, "mxfp4")
+    x = [[bf16(b) for b in row] for row in X]
+    B = []
+    for row in x:
+        out = []
+        for g0 in range(0, K, 4):
+            kp = keep_top2(row[g0:g0 + 4])
+            out += [row[g0 + i] if i in kp else Fraction(0) for i in range(4)]
+        B.append(out)
+    bc, bs, bd = model_mxfp4(B)
+    assert [pack(r) for r in bc] == R.bb.codes.tolist() and bs == R.bb.scales.tolist()
+    res = [[rne32(v - d) for v, d in zip(row, drow)] for row, drow in zip(x, bd)]
+    rc, rs, _ = model_mxfp4(res)
+    assert [pack(r) for r in rc] == R.rs.codes.tolist()
+    assert rs == R.rs.scales.tolist()
+    assert float(R.rs.tscale) == 1.0
+
+
+def test_nvfp4_shared_residual_chain_is_the_exact_model():
+    """Shared residual scale: the residual's quantiser takes the backbone's
+    tensor maximum A_b, so its G_enc, k1 and G_dec are the backbone's."""
+    M, K = 2, 256
+    X = wl.activation("student_t", 101, 0, M, K)
+    R = oracle.prepare(X, None, 1e-6, 2, 4, "nvfp4", residual_scale="shared")
+    x = [[bf16(b) for b in row] for row in X]
+    B = []
+    for row in x:
+        out = []
+        for g0 in range(0, K, 4):
+            kp = keep_top2(row[g0:g0 + 4])
+            out += [row[g0 + i] if i in kp else Fraction(0) for i in range(4)]
+        B.append(out)
+    A_b = max(abs(v) for row in x for v in row)
+    bc, bs, bgdec = model_nvfp4(B, A_b)
+    assert [pack(r) for r in bc] == R.bb.codes.tolist()
+    res = []
+    for i, row in enumerate(x):
+        rr = []
+        for k, v in enumerate(row):
+            c = bc[i][k]
+            d = rne32(rne32((-1 if c & 8 else 1) * E2M1[c & 7] * E4M3[bs[i][k // 16]]) * bgdec)
+            rr.append(rne32(v - d))
+        res.append(rr)
+    rcodes, rscales, rgdec = model_nvfp4(res, A_b)
+    assert [pack(r) for r in rcodes] == R.rs.codes.tolist()
+    assert rscales == R.rs.scales.tolist()
+    assert Fraction(float(R.rs.tscale)) == rgdec == bgdec
+
+
+def test_pair_prepare_chain_is_the_exact_model():
+    """Pair-granular 4:8 prepare with RMSNorm: y on the exact model, pair
+    magnitude max(|y_2i|, |y_2i+1|), the two strongest of four pairs kept
+    (ties to the lower pair), MXFP4 backbone and residual, and the
+    compressed form: the kept pairs' code bytes in order and one nibble per
+    group of eight (lower kept pair index in bits 1:0), group 2j in the low
+    nibble of byte j."""
+    M, K = 2, 256
+    X = wl.activation("laplace_outlier", 102, 0, M, K)
+    g = wl.gamma_random(102, 0, K)
+    P, kept, meta = oracle.prepare_pairs(X, g, 1e-6)
+    ys, B, nibs = [], [], []
+    for row in X:
+        r = model_rinv(row, 1e-6)
+        y = [rne32(rne32(bf16(xv) * r) * bf16(gk)) for xv, gk in zip(row, g)]
+        ys.append(y)
+        out, rn = [], []
+        for g0 in range(0, K, 8):
+            mag = [max(abs(y[g0 + 2 * p]), abs(y[g0 + 2 * p + 1])) for p in range(4)]
+            order = sorted(range(4), key=lambda p: (-mag[p], p))
+            lo, hi = sorted(order[:2])
+            rn.append(lo | (hi << 2))
+            out += [y[g0 + i] if i // 2 in (lo, hi) else Fraction(0) for i in range(8)]
+        B.append(out)
+        nibs.append(rn)
+    bc, bs, bd = model_mxfp4(B)
+    assert [pack(r) for r in bc] == P.bb.codes.tolist() and bs == P.bb.scales.tolist()
+    for i in range(M):
+        packed = pack(bc[i])
+        want_kept = []
+        for gi, nb in enumerate(nibs[i]):
+            want_kept += [packed[4 * gi + (nb & 3)], packed[4 * gi + (nb >> 2)]]
+        assert want_kept == kept[i].tolist()
+        want_meta = [nibs[i][2 * j] | (nibs[i][2 * j + 1] << 4) for j in range(K // 16)]
+        assert want_meta == meta[i].tolist()
+    res = [[rne32(v - d) for v, d in zip(row, drow)] for row, drow in zip(ys, bd)]
+    rc, rs, _ = model_mxfp4(res)
+    assert [pack(r) for r in rc] == P.rs.codes.tolist() and rs == P.rs.scales.tolist()
