@@ -450,3 +450,31 @@ def test_residual_tensor_max_is_pruned_or_kept_max(dist, gk):
         assert P >= Q
     else:
         assert Q > P
+
+
+def test_bf16_rne_reference_against_exact_rounding():
+    """RNE(Y64) to bf16 against a brute-force nearest-even choice on exact
+    rationals, on random values and on values a hair off bf16 midpoints
+    (where a rounding through fp32 first would land on the midpoint and
+    then tie the wrong way)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    base = rng.standard_normal(400) * 10.0 ** rng.integers(-6, 6, 400)
+    mids = []
+    for b in rng.integers(0x3000, 0x4F00, 200).astype(np.uint32):
+        lo = float((b << np.uint32(16)).view(np.float32))
+        hi = float(((b + np.uint32(1)) << np.uint32(16)).view(np.float32))
+        mid = (lo + hi) / 2
+        for d in (-1e-13, 1e-13, 0.0):
+            mids += [mid * (1 + d), -mid * (1 + d)]
+    Y = np.concatenate([base, np.array(mids)])
+    got = oracle.bf16_rne_from_f64(Y)
+    for y, g in zip(Y, got):
+        q = Fraction(float(y))
+        b32 = np.array([y], dtype=np.float32).view(np.uint32)[0] >> np.uint32(16)
+        cands = [int(b32) + k for k in (-2, -1, 0, 1, 2) if 0 <= int(b32) + k < 0xFFFF]
+        def val(c):
+            return Fraction(float((np.uint32(c) << np.uint32(16)).view(np.float32)))
+        cands = [c for c in cands if np.isfinite(float(val(c)))]
+        best = min(cands, key=lambda c: (abs(val(c) - q), c & 1))
+        assert int(g) == best, (y, hex(int(g)), hex(best))
