@@ -116,3 +116,24 @@ def test_moe_swiglu_is_the_per_expert_loop():
         e = int(np.searchsorted(off, t, side="right") - 1)
         want = oracle.swiglu_linear(oracle.gather_rows(P, ri[t:t + 1]), Wq[e])[0]
         np.testing.assert_array_equal(H[t], want)
+
+
+def test_moe_swiglu_parts_are_the_per_row_parts():
+    """All four grouped parts (gate, up and their magnitude-sum bounds, which
+    set the grouped SwiGLU test's tolerance) equal the plain parts of each
+    dispatched row through its own expert."""
+    T_tok, E, K, I = 10, 4, 256, 64
+    X = wl.activation("laplace_outlier", 94, 0, T_tok, K)
+    P = oracle.prepare(X, wl.gamma_ones(K), 1e-6, 2, 4, "nvfp4")
+    ex = np.zeros((T_tok, 2), dtype=np.int32)
+    ex[:, 1] = 3
+    ex[:4, 0] = 1                                   # expert 2 empty
+    ri, off = wl.group_by_expert(ex, E)
+    Wq = [oracle.quantize_weight(oracle.interleave_gate_up(wl.weight(94, 10 + e, I, K),
+                                                           wl.weight(94, 20 + e, I, K))) for e in range(E)]
+    parts = oracle.moe_swiglu_parts(P, ri, off, Wq)
+    for t in range(len(ri)):
+        e = int(np.searchsorted(off, t, side="right") - 1)
+        want = oracle.swiglu_parts(oracle.gather_rows(P, ri[t:t + 1]), Wq[e])
+        for got, w in zip(parts, want):
+            np.testing.assert_array_equal(got[t], w[0])
