@@ -122,6 +122,43 @@ def test_prepare_layernorm_bit_exact(M, K, dist, hb, n, m, fmt, rs):
     assert to_np(P.rs_tscale).view(np.uint32)[0] == np.float32(R.rs.tscale).view(np.uint32)
 
 
+# Long rows: gamma (and beta) no longer fit the kernel's 96 KiB shared-memory
+# stage and are read from global memory (RMSNorm K > 24576, LayerNorm with a
+# bias K > 12288), and MXFP4 RMSNorm rows past the 4096 elements it holds in
+# registers take the chunked path.
+LONG_K_CASES = [
+    # M, K, norm, beta, fmt, residual
+    (5, 32768, "rms", False, "nvfp4", "own"),
+    (3, 32768, "rms", False, "mxfp4", "own"),
+    (9, 8192, "rms", False, "mxfp4", "own"),
+    (4, 32768, "rms", False, "nvfp4", "shared"),
+    (7, 16384, "layernorm", True, "nvfp4", "own"),
+    (6, 32768, "layernorm", False, "mxfp4", "own"),
+]
+
+
+@pytest.mark.parametrize("M,K,norm,hb,fmt,rs", LONG_K_CASES)
+def test_prepare_long_rows_bit_exact(M, K, norm, hb, fmt, rs):
+    X = wl.activation("laplace_outlier", 27, M + K, M, K)
+    g = wl.gamma_random(27, 0, K)
+    if norm == "rms":
+        run_and_compare(X, g, 2, 4, fmt, residual_scale=rs)
+        return
+    b = wl.beta_random(27, 0, K) if hb else None
+    P = sq.prepare_layernorm(to_dev(X), to_dev(g), None if b is None else to_dev(b), 1e-6, 2, 4, fmt,
+                             want_mask=True, residual_scale=rs)
+    torch.cuda.synchronize()
+    assert sq.last_device_status() == 0
+    R = oracle.prepare(X, g, 1e-6, 2, 4, fmt, residual_scale=rs, norm="layernorm", beta=b)
+    assert np.array_equal(to_np(P.mask), R.mask), "mask"
+    assert np.array_equal(to_np(P.bb_codes), R.bb.codes), "backbone codes"
+    assert np.array_equal(to_np(P.rs_codes), R.rs.codes), "residual codes"
+    assert np.array_equal(atoms_to_canonical(to_np(P.bb_scales), M, K, fmt), R.bb.scales)
+    assert np.array_equal(atoms_to_canonical(to_np(P.rs_scales), M, K, fmt), R.rs.scales)
+    assert to_np(P.bb_tscale).view(np.uint32)[0] == np.float32(R.bb.tscale).view(np.uint32)
+    assert to_np(P.rs_tscale).view(np.uint32)[0] == np.float32(R.rs.tscale).view(np.uint32)
+
+
 def test_prepare_layernorm_constant_rows_give_beta():
     """Constant rows normalise to exactly beta: the backbone and residual
     are those of the tensor [beta; beta; ...] with no norm."""
